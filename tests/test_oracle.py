@@ -1,0 +1,413 @@
+"""Pins for the fp64 oracle, checked against things other than itself:
+
+* the attention tutorial page's worked examples (tests/golden/),
+* the tau -> 0 limit, which the MALA paper's cost paragraph says recovers
+  FullAttn: dense masked softmax and its autograd gradient (torch, fp64),
+* brute force on tiny inputs in the paper's *ratio* form (explicit retained
+  key sets, plain exponentials) rather than the oracle's log form,
+* invariants stated in the paper: m + log l = log Z over the retained set,
+  the contribution ratio upper-bounds the dense probability, backward
+  support nests inside forward support, the first legal tile is retained,
+* closed forms: tau = inf keeps only the diagonal tile; decode with one split
+  equals the causal forward of the last row; split merge at tau = 0 equals
+  the dense softmax.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import mala_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_golden(name):
+    rows = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, _, rest = line.partition(" ")
+            rows[key] = rest
+    return rows
+
+
+def _nums(s):
+    return [float(x) for x in s.split()]
+
+
+def _rand_case(seed, N, d, H=1, sharp=2.0):
+    rng = np.random.default_rng(seed)
+    Q = rng.standard_normal((N, d)) * sharp / math.sqrt(d)
+    K = rng.standard_normal((N, d))
+    V = rng.standard_normal((N, d))
+    return Q, K, V
+
+
+def _dense_torch(Q, K, V):
+    """Dense causal masked softmax attention in fp64 (the tutorial page's
+    teaching reference, masked before the softmax)."""
+    q = torch.tensor(Q, dtype=torch.float64, requires_grad=True)
+    k = torch.tensor(K, dtype=torch.float64, requires_grad=True)
+    v = torch.tensor(V, dtype=torch.float64, requires_grad=True)
+    N = q.shape[0]
+    s = q @ k.T
+    allowed = torch.tril(torch.ones(N, N, dtype=torch.bool))
+    s = s.masked_fill(~allowed, -float("inf"))
+    w = torch.softmax(s, dim=-1)
+    out = w @ v
+    lse = torch.logsumexp(s, dim=-1)
+    return q, k, v, out, lse, w
+
+
+# ---------------------------------------------------------------- golden
+
+def test_masked_row_worked_example():
+    g = _read_golden("masked_row.txt")
+    raw = _nums(g["raw_products"])
+    dk = float(g["d_k"])
+    scaled = _nums(g["scaled_scores"])
+    qpos = int(g["query_position"])
+    fut = int(g["future_keys"])
+    assert np.allclose(np.array(raw) / math.sqrt(dk), scaled)
+    # Q row qpos carries the scaled products against K = identity, V = identity
+    N = 4
+    Q = np.zeros((N, 4))
+    Q[qpos] = scaled
+    K = np.eye(4)
+    V = np.eye(4)
+    O, z, keep, _ = orc.forward_head(Q, K, V, 1, 1, 0.0)
+    w = O[qpos]                                   # weights, since V = I
+    assert w[fut] == 0.0                          # future key: exactly zero
+    assert abs(w.sum() - 1.0) < 1e-15
+    e = np.exp(np.array(scaled[:qpos + 1]))
+    assert np.allclose(w[:qpos + 1], e / e.sum(), rtol=0, atol=1e-15)
+    assert abs(z[qpos] - math.log(e.sum())) < 1e-14
+
+
+def test_online_accumulator_worked_example():
+    g = _read_golden("online_accumulator.txt")
+    s = _nums(g["scores"])
+    vals = np.array([_nums(t) for t in g["values"].split(";")])
+    run_max = _nums(g["running_max"])
+    # one query at position 3 sees all four keys; K = identity carries the
+    # scores; one key per tile, visited in the page's order 0, 1, 2, 3
+    q = np.array(s)[None, :]
+    K = np.eye(4)
+    seen = []
+    st = orc.forward_block(q, np.array([3]), K, vals, 1, 0.0, [0, 1, 2, 3],
+                           trace=lambda j, x: seen.append(x))
+    assert [x["m"][0] for x in seen] == run_max
+    # after tile 2 the first tile's weight is expressed relative to max 3
+    assert abs(seen[1]["l"][0] - (math.exp(-3.0) + 1.0)) < 1e-15
+    O, z = orc.finalize(st)
+    e = np.exp(np.array(s))
+    assert np.allclose(O[0], (e / e.sum()) @ vals, atol=1e-15)
+
+
+# ---------------------------------------------------------------- tau -> 0
+
+@pytest.mark.parametrize("N,d,Bq,Bk", [(37, 8, 8, 8), (33, 4, 4, 8), (40, 6, 16, 4), (17, 3, 1, 1)])
+def test_tau_zero_is_dense_attention(N, d, Bq, Bk):
+    Q, K, V = _rand_case(N * 7 + d, N, d, sharp=3.0)
+    O, z, keep, margin = orc.forward_head(Q, K, V, Bq, Bk, 0.0)
+    _, _, _, out, lse, _ = _dense_torch(Q, K, V)
+    assert np.abs(O - out.detach().numpy()).max() < 1e-12
+    assert np.abs(z - lse.detach().numpy()).max() < 1e-12
+    # every legal tile retained
+    for i in range(keep.shape[0]):
+        last = min((i + 1) * Bq, N) - 1
+        assert keep[i, : last // Bk + 1].all()
+        assert not keep[i, last // Bk + 1:].any()
+
+
+@pytest.mark.parametrize("N,d,Bq,Bk", [(23, 5, 4, 4), (30, 4, 8, 4), (19, 3, 4, 8)])
+def test_tau_zero_backward_is_dense_gradient(N, d, Bq, Bk):
+    Q, K, V = _rand_case(N * 3 + d, N, d, sharp=3.0)
+    dO = np.random.default_rng(N).standard_normal((N, d))
+    q, k, v, out, lse, _ = _dense_torch(Q, K, V)
+    out.backward(torch.tensor(dO))
+    O, z, keep, _ = orc.forward_head(Q, K, V, Bq, Bk, 0.0)
+    dQ, dK, dV, bkeep, _ = orc.backward_head(Q, K, V, O, dO, z, Bq, Bk, 0.0, keep)
+    assert np.abs(dQ - q.grad.numpy()).max() < 1e-11
+    assert np.abs(dK - k.grad.numpy()).max() < 1e-11
+    assert np.abs(dV - v.grad.numpy()).max() < 1e-11
+    # pure (mask-free) backward gives the same at tau = 0
+    dQ2, dK2, dV2, _, _ = orc.backward_head(Q, K, V, O, dO, z, Bq, Bk, 0.0, None)
+    assert np.abs(dQ2 - dQ).max() < 1e-13 and np.abs(dK2 - dK).max() < 1e-13
+
+
+def test_gqa_backward_sums_group():
+    rng = np.random.default_rng(5)
+    B, N, Hq, Hkv, d = 1, 12, 4, 2, 4
+    q = rng.standard_normal((B, N, Hq, d))
+    k = rng.standard_normal((B, N, Hkv, d))
+    v = rng.standard_normal((B, N, Hkv, d))
+    do = rng.standard_normal((B, N, Hq, d))
+    O, lse, keep, _ = orc.forward(q, k, v, 4, 4, 0.0)
+    dq, dk, dv, _ = orc.backward(q, k, v, O, do, lse, 4, 4, 0.0, keep)
+    qt = torch.tensor(q, requires_grad=True)
+    kt = torch.tensor(k, requires_grad=True)
+    vt = torch.tensor(v, requires_grad=True)
+    ke = kt.repeat_interleave(2, dim=2)
+    ve = vt.repeat_interleave(2, dim=2)
+    s = torch.einsum("bqhd,bkhd->bhqk", qt, ke)
+    s = s.masked_fill(~torch.tril(torch.ones(N, N, dtype=torch.bool)), -float("inf"))
+    out = torch.einsum("bhqk,bkhd->bqhd", torch.softmax(s, -1), ve)
+    out.backward(torch.tensor(do))
+    assert np.abs(O - out.detach().numpy()).max() < 1e-12
+    assert np.abs(dq - qt.grad.numpy()).max() < 1e-11
+    assert np.abs(dk - kt.grad.numpy()).max() < 1e-11
+    assert np.abs(dv - vt.grad.numpy()).max() < 1e-11
+
+
+# ---------------------------------------------------------------- brute force
+
+def _brute_forward(Q, K, V, Bq, Bk, tau):
+    """The paper's test in ratio form with explicit retained key sets:
+    r_qj = max_{k in J_j, legal} exp(s_qk) / sum_{k in R_q} exp(s_qk);
+    skip iff r < tau / L_q for every row with a legal key (empty R: keep)."""
+    N = Q.shape[0]
+    S = Q @ K.T
+    nQB, nKB = -(-N // Bq), -(-N // Bk)
+    keep = np.zeros((nQB, nKB), dtype=bool)
+    O = np.zeros_like(V)
+    for i in range(nQB):
+        rows = list(range(i * Bq, min((i + 1) * Bq, N)))
+        R = {q: [] for q in rows}
+        for j in range(min(rows[-1] // Bk, nKB - 1), -1, -1):
+            cols = list(range(j * Bk, min((j + 1) * Bk, N)))
+            retain = False
+            for q in rows:
+                legal = [k for k in cols if k <= q]
+                if not legal:
+                    continue
+                if not R[q]:
+                    retain = True
+                    continue
+                Z = sum(math.exp(S[q, k]) for k in R[q])
+                r = max(math.exp(S[q, k]) for k in legal) / Z
+                if not (r < tau / (q + 1)):
+                    retain = True
+            keep[i, j] = retain
+            if retain:
+                for q in rows:
+                    R[q] += [k for k in cols if k <= q]
+        for q in rows:
+            w = np.array([math.exp(S[q, k]) for k in R[q]])
+            O[q] = (w / w.sum()) @ V[R[q]]
+    return keep, O
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("tau", [0.05, 0.3, 1.0, 4.0])
+def test_forward_matches_brute_force(seed, tau):
+    rng = np.random.default_rng(seed)
+    N = int(rng.integers(9, 33))
+    d = int(rng.integers(2, 9))
+    Bq = int(rng.choice([1, 2, 4, 8]))
+    Bk = int(rng.choice([1, 2, 4, 8]))
+    Q, K, V = _rand_case(100 + seed, N, d, sharp=4.0)
+    keep_b, O_b = _brute_forward(Q, K, V, Bq, Bk, tau)
+    O, z, keep, margin = orc.forward_head(Q, K, V, Bq, Bk, tau)
+    assert (keep == keep_b).all()
+    assert np.abs(O - O_b).max() < 1e-12
+    # decisions are not degenerate across the parametrisation
+    visited = ~np.isnan(margin)
+    assert visited.sum() >= keep.sum() > 0
+
+
+def test_brute_force_sees_skips():
+    """Make sure the brute-force comparison actually exercises skipping."""
+    Q, K, V = _rand_case(7, 32, 8, sharp=6.0)
+    keep, _ = _brute_forward(Q, K, V, 4, 4, 1.0)
+    legal = sum(min((i * 4 + 3) // 4, 7) + 1 for i in range(8))
+    assert 0 < keep.sum() < legal
+
+
+def _brute_backward(Q, K, V, O, dO, z, Bq, Bk, tau, fwd_keep):
+    """Dense (untiled) restatement of the backward: an entry contributes iff
+    its tile was forward-retained and some legal entry of the tile has
+    probability exp(s - z) >= tau / L_q."""
+    N = Q.shape[0]
+    S = Q @ K.T
+    P = np.zeros((N, N))
+    E = np.zeros((N, N), dtype=bool)
+    for i in range(fwd_keep.shape[0]):
+        for j in range(fwd_keep.shape[1]):
+            if not fwd_keep[i, j]:
+                continue
+            rows = range(i * Bq, min((i + 1) * Bq, N))
+            cols = range(j * Bk, min((j + 1) * Bk, N))
+            ent = [(q, k) for q in rows for k in cols if k <= q]
+            if not ent:
+                continue
+            if any(math.exp(S[q, k] - z[q]) >= tau / (q + 1) for (q, k) in ent):
+                for (q, k) in ent:
+                    E[q, k] = True
+    P[E] = np.exp(S - z[:, None])[E]
+    D = (dO * O).sum(1)
+    dV = P.T @ dO
+    dP = dO @ V.T
+    dS = np.where(E, P * (dP - D[:, None]), 0.0)
+    return dS @ K, dS.T @ Q, dV
+
+
+@pytest.mark.parametrize("seed", range(5))
+@pytest.mark.parametrize("tau", [0.1, 1.0])
+def test_backward_matches_brute_force(seed, tau):
+    rng = np.random.default_rng(50 + seed)
+    N = int(rng.integers(9, 29))
+    d = int(rng.integers(2, 7))
+    Bq = int(rng.choice([2, 4, 8]))
+    Bk = int(rng.choice([2, 4, 8]))
+    Q, K, V = _rand_case(200 + seed, N, d, sharp=4.0)
+    dO = rng.standard_normal((N, d))
+    O, z, keep, _ = orc.forward_head(Q, K, V, Bq, Bk, tau)
+    dQ, dK, dV, bkeep, _ = orc.backward_head(Q, K, V, O, dO, z, Bq, Bk, tau, keep)
+    bq, bk, bv = _brute_backward(Q, K, V, O, dO, z, Bq, Bk, tau, keep)
+    assert np.abs(dQ - bq).max() < 1e-12
+    assert np.abs(dK - bk).max() < 1e-12
+    assert np.abs(dV - bv).max() < 1e-12
+
+
+# ---------------------------------------------------------------- invariants
+
+@pytest.mark.parametrize("tau", [0.02, 0.5, 2.0])
+def test_lse_invariant_and_ratio_bound(tau):
+    """m + log l = log Z over the retained set after every tile, and the
+    contribution ratio upper-bounds the dense probability of the tile."""
+    N, d, B = 48, 8, 8
+    Q, K, V = _rand_case(11, N, d, sharp=5.0)
+    S = Q @ K.T
+    lse_dense = np.array([np.log(np.exp(S[q, :q + 1]).sum()) for q in range(N)])
+    for i in range(N // B):
+        rows = np.arange(i * B, (i + 1) * B)
+        retained = {int(q): [] for q in rows}
+        prev = {}
+
+        def check(j, st):
+            cols = np.arange(j * B, (j + 1) * B)
+            for r, q in enumerate(rows):
+                legal = cols[cols <= q]
+                if len(legal) == 0:
+                    continue
+                # the ratio bound uses the state *before* this tile's update
+                if q in prev and prev[q][1] > 0:
+                    m0, l0 = prev[q]
+                    ratio = math.exp(S[q, legal].max() - m0) / l0
+                    p_dense = math.exp(S[q, legal].max() - lse_dense[q])
+                    assert ratio >= p_dense * (1 - 1e-12)
+                if st["keep"]:
+                    retained[int(q)] += list(legal)
+                if retained[int(q)]:
+                    logZ = np.log(np.exp(S[q, retained[int(q)]]).sum())
+                    assert abs(st["m"][r] + math.log(st["l"][r]) - logZ) < 1e-12
+                prev[q] = (st["m"][r], st["l"][r])
+
+        orc.forward_block(Q[rows], rows, K, V, B, tau,
+                          orc.causal_tiles(rows[-1], B, N // B), trace=check)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_backward_support_nests_in_forward(seed):
+    Q, K, V = _rand_case(300 + seed, 64, 8, sharp=5.0)
+    dO = np.random.default_rng(seed).standard_normal((64, 8))
+    for tau in (0.05, 0.5, 2.0):
+        O, z, keep, _ = orc.forward_head(Q, K, V, 8, 8, tau)
+        _, _, _, pure_keep, pure_margin = orc.backward_head(Q, K, V, O, dO, z, 8, 8, tau, None)
+        bad = pure_keep & ~keep
+        assert not bad.any() or np.abs(pure_margin[bad]).max() < 1e-9
+
+
+def test_first_legal_tile_always_retained():
+    Q, K, V = _rand_case(9, 40, 4, sharp=8.0)
+    for tau in (0.5, 5.0, 1e6):
+        _, _, keep, _ = orc.forward_head(Q, K, V, 8, 8, tau)
+        for i in range(5):
+            assert keep[i, i]
+
+
+def test_tau_infinite_keeps_only_diagonal():
+    N, d, B = 32, 4, 8
+    Q, K, V = _rand_case(21, N, d, sharp=2.0)
+    O, z, keep, _ = orc.forward_head(Q, K, V, B, B, math.inf)
+    assert (keep == np.eye(N // B, dtype=bool)).all()
+    S = Q @ K.T
+    for q in range(N):
+        k0 = (q // B) * B
+        w = np.exp(S[q, k0:q + 1] - S[q, k0:q + 1].max())
+        assert np.allclose(O[q], (w / w.sum()) @ V[k0:q + 1], atol=1e-13)
+    dO = np.ones((N, d))
+    dQ, dK, dV, bkeep, _ = orc.backward_head(Q, K, V, O, dO, z, B, B, math.inf, keep)
+    assert not bkeep.any() and not dQ.any() and not dK.any() and not dV.any()
+
+
+def test_sharper_tau_skips_more_and_omits_more_mass():
+    Q, K, V = _rand_case(31, 64, 8, sharp=4.0)
+    _, z0, k0, _ = orc.forward_head(Q, K, V, 8, 8, 0.0)
+    prev_kept, prev_mass = k0.sum(), 0.0
+    for tau in (0.01, 0.1, 1.0):
+        _, z, kp, _ = orc.forward_head(Q, K, V, 8, 8, tau)
+        omitted = 1.0 - np.exp(z - z0)          # paper's omitted-mass metric
+        assert (omitted >= -1e-12).all()
+        assert kp.sum() <= prev_kept
+        prev_kept = kp.sum()
+
+
+# ---------------------------------------------------------------- decode
+
+def test_decode_single_split_equals_last_causal_row():
+    rng = np.random.default_rng(3)
+    N, d, Bk = 8 * 5 + 1, 6, 8                     # last query block holds one row
+    Q = rng.standard_normal((N, d)) * 3 / math.sqrt(d)
+    K = rng.standard_normal((N, d))
+    V = rng.standard_normal((N, d))
+    for tau in (0.0, 0.1, 1.0):
+        O, z, keep, margin = orc.forward_head(Q, K, V, 8, Bk, tau)
+        Od, zd, kd, md, _ = orc.decode_head(Q[-1], K, V, Bk, tau, 1)
+        assert np.allclose(Od, O[-1], atol=1e-14) and abs(zd - z[-1]) < 1e-14
+        assert (kd == keep[-1]).all()
+
+
+@pytest.mark.parametrize("P", [1, 2, 3, 7])
+def test_decode_splits_at_tau_zero_are_dense(P):
+    rng = np.random.default_rng(P)
+    N, d, Bk = 61, 5, 8
+    q = rng.standard_normal(d)
+    K = rng.standard_normal((N, d))
+    V = rng.standard_normal((N, d))
+    O, z, keep, _, parts = orc.decode_head(q, K, V, Bk, 0.0, P)
+    s = K @ q
+    w = np.exp(s - s.max())
+    assert np.allclose(O, (w / w.sum()) @ V, atol=1e-13)
+    assert abs(z - (s.max() + math.log(w.sum()))) < 1e-13
+    assert keep.all() and len(parts) == P
+
+
+def test_decode_first_tile_of_each_split_retained():
+    rng = np.random.default_rng(4)
+    N, d, Bk, P = 128, 4, 8, 4
+    q = rng.standard_normal(d) * 4
+    K = rng.standard_normal((N, d))
+    V = rng.standard_normal((N, d))
+    _, _, keep, _, _ = orc.decode_head(q, K, V, Bk, math.inf, P)
+    for (t0, t1) in orc.split_ranges(N // Bk, P):
+        assert keep[t1 - 1]
+        assert not keep[t0:t1 - 1].any()
+    assert orc.split_ranges(10, 3) == [(0, 3), (3, 6), (6, 10)]
+
+
+def test_replay_forces_decisions_but_keeps_margins():
+    Q, K, V = _rand_case(41, 32, 4, sharp=5.0)
+    O, z, keep, margin = orc.forward_head(Q, K, V, 8, 8, 0.5)
+    O2, z2, keep2, margin2 = orc.forward_head(Q, K, V, 8, 8, 0.5, replay_mask=keep)
+    assert (keep2 == keep).all() and np.allclose(O2, O) and np.allclose(margin2, margin, equal_nan=True)
+    flipped = keep.copy()
+    flipped[3, 1] = not flipped[3, 1]
+    _, _, keep3, _ = orc.forward_head(Q, K, V, 8, 8, 0.5, replay_mask=flipped)
+    assert keep3[3, 1] == flipped[3, 1]
