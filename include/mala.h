@@ -1,0 +1,232 @@
+/*
+ * mala.h - C ABI of the MassAlloc Attention (MALA) operator library for B200.
+ *
+ * Source of the operation: "MassAlloc Attention: Let Attention Allocate Its
+ * Own Compute", method section. Run-in headings cited below:
+ *   "Setup"                       problem statement: Q [N_q, d], K/V [N_k, d],
+ *                                 1/sqrt(d) folded into Q, natural exp/log,
+ *                                 query blocks I_i of B_q rows, key blocks J_j
+ *                                 of B_k rows, L_q = |C_q|, threshold tau/L_q;
+ *                                 L_q = q + 1 in training, L_0 = N_k in
+ *                                 single-token decoding.
+ *   "Online Sparse Softmax"       forward skip test (Algorithm 1).
+ *   "Offline Sparse Probability"  backward skip test (Algorithm 2).
+ *   Appendix A.1                  fused forward / backward / decoding
+ *                                 execution and traversal orders.
+ * Tensor layout follows the FlashAttention interface on the attention
+ * tutorial page ("Hardware paths and kernel contracts"): Q, O, dQ, dO are
+ * [B, N_q, H_q, d]; K, V, dK, dV are [B, N_k, H_kv, d]; the last dimension
+ * is contiguous and the other strides are passed in elements.
+ *
+ * Conventions common to every entry point
+ *   - All tensor pointers are caller-owned DEVICE memory. The library never
+ *     allocates or frees memory; scratch space is the caller's `workspace`
+ *     buffer of at least mala_*_workspace_size() bytes (NULL allowed when
+ *     that size is 0).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Arguments are checked on the host before anything is
+ *     launched; on a non-zero return nothing was launched.
+ *   - Scale: the caller folds 1/sqrt(d) into Q; gradients are with respect
+ *     to the scaled Q.
+ *   - tau >= 0. tau = 0 skips nothing (FullAttn); tau = +inf retains only
+ *     the first legal tile of every query block / split.
+ *   - Query head h reads key/value head q_to_kv[h] (a HOST array of H_q
+ *     entries, copied during the call); NULL means h / (H_q / H_kv).
+ *   - keep masks are uint32 bit sets: bit (j % 32) of word j / 32 of the
+ *     row for (b, h, i) is set iff tile (i, j) was retained.
+ *   - Kernels never trap. A device-side bounded wait that gives up records
+ *     MALA_ERR_TIMEOUT, which mala_check_device_error() reports.
+ */
+#ifndef MALA_H_
+#define MALA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MALA_API __attribute__((visibility("default")))
+#else
+#define MALA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+enum {
+  MALA_OK = 0,
+  MALA_ERR_INVALID_ARG = 1,   /* NULL pointer, bad size/stride/alignment, tau < 0 or NaN */
+  MALA_ERR_UNSUPPORTED = 2,   /* valid request this build has no kernel for */
+  MALA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+  MALA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  MALA_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up */
+};
+
+/* element types of Q, K, V, O (and dO, dQ, dK, dV) */
+enum { MALA_BF16 = 0, MALA_FP32 = 1 };
+
+/* masking mode of mala_fwd */
+enum {
+  MALA_CAUSAL = 0,  /* N_q = N_k, key k legal for row q iff k <= q, L_q = q + 1 */
+  MALA_DECODE = 1   /* reserved for mala_fwd: single-token decoding uses mala_decode */
+};
+
+/*
+ * Forward / prefill: Algorithm 1 ("Online Sparse Softmax", Appendix A.1
+ * "Fused forward execution"). For every query block, every legal key tile is
+ * scored (S_ij = Q_i K_j^T), key blocks visited in descending order from the
+ * diagonal. A tile is skipped iff, for every valid row q with a legal key in
+ * it, max_k s_qk - (m_q + log l_q) < log tau - log L_q; a row whose retained
+ * set is empty always retains. Only retained tiles load V and run the
+ * online-softmax update and PV.
+ *
+ * Outputs: o [B, N_q, H_q, d] (same dtype as q) = softmax renormalised over
+ * the retained tiles; lse [B, H_q, N_q] fp32 = z_q = m_q + log l_q (natural
+ * log), the state the backward pass consumes; keep_mask (optional, may be
+ * NULL) [B, H_q, ceil(N_q/B_q), ceil(ceil(N_k/B_k)/32)] uint32; stats
+ * (optional device int64[4], accumulated with atomics, caller zeroes):
+ * tiles tested, tiles retained, post-score key slots (B_k per row per
+ * retained tile, valid rows only), reserved.
+ *
+ * Supported: dtype MALA_BF16 with d in {64, 128} and B_q = B_k = 128 (tensor
+ * core path); dtype MALA_FP32 or MALA_BF16 with d in {64, 128} and
+ * B_q, B_k in {16, 32, 64, 128} (CUDA-core path). mode MALA_CAUSAL only.
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  uint32_t* keep_mask;
+  int64_t batch, heads_q, heads_kv, seqlen_q, seqlen_k, head_dim;
+  int64_t q_stride[3];          /* batch, sequence, head strides in elements */
+  int64_t k_stride[3];
+  int64_t v_stride[3];
+  int64_t o_stride[3];
+  const int32_t* q_to_kv;       /* host array [heads_q] or NULL */
+  int32_t block_q, block_k;
+  float tau;
+  int32_t dtype;
+  int32_t mode;
+  int64_t* stats;               /* device int64[4] or NULL */
+} mala_fwd_args;
+
+MALA_API size_t mala_fwd_workspace_size(const mala_fwd_args* args);
+MALA_API int mala_fwd(const mala_fwd_args* args, void* workspace, size_t workspace_bytes,
+             void* stream);
+
+/*
+ * Backward: Algorithm 2 ("Offline Sparse Probability", Appendix A.1 "Fused
+ * backward execution"). Key-major: for every key block j, query blocks are
+ * visited ascending from the diagonal; the score tile is recomputed and the
+ * tile is skipped iff s_qk - z_q < log tau - log L_q for every legal (q, k)
+ * entry, z = lse from mala_fwd. Retained tiles reconstruct P = exp(S - z)
+ * and run dV += P^T dO, dP = dO V^T, dS = P * (dP - D) with
+ * D_q = sum_d dO_q O_q, dQ += dS K, dK += dS^T Q. dK and dV of a key/value
+ * head sum the contributions of every query head mapped to it.
+ *
+ * keep_mask (input, optional): the forward's mask. When given, only tiles
+ * the forward retained are recomputed (mask replay; by the support-nesting
+ * argument of the same section this selects the same tiles up to rounding).
+ * NULL visits every legal tile. bwd_keep_mask (output, optional): same
+ * layout, bits of tiles the backward retained. dq, dk, dv are fully
+ * overwritten. Supported: MALA_BF16, d = 128, B_q = B_k = 128.
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;
+  const uint32_t* keep_mask;
+  void* dq;
+  void* dk;
+  void* dv;
+  uint32_t* bwd_keep_mask;
+  int64_t batch, heads_q, heads_kv, seqlen_q, seqlen_k, head_dim;
+  int64_t q_stride[3];
+  int64_t k_stride[3];
+  int64_t v_stride[3];
+  int64_t o_stride[3];
+  int64_t do_stride[3];
+  int64_t dq_stride[3];
+  int64_t dk_stride[3];
+  int64_t dv_stride[3];
+  const int32_t* q_to_kv;
+  int32_t block_q, block_k;
+  float tau;
+  int32_t dtype;
+  int64_t* stats;               /* device int64[4]: tiles tested, retained, slots, reserved */
+} mala_bwd_args;
+
+MALA_API size_t mala_bwd_workspace_size(const mala_bwd_args* args);
+MALA_API int mala_bwd(const mala_bwd_args* args, void* workspace, size_t workspace_bytes,
+             void* stream);
+
+/*
+ * Single-token decoding with split-KV (cost paragraph after "Offline Sparse
+ * Probability"; Appendix A.1 "Fused decoding execution"). One query per
+ * (batch, head) at position N_k - 1, so L_0 = N_k. The T = ceil(N_k/B_k) key
+ * tiles are split into P contiguous ranges, split p covering tiles
+ * [floor(p*T/P), floor((p+1)*T/P)); each split visits its tiles in
+ * descending order with its own running maximum and normalisation sum, and
+ * tests every tile against tau / N_k. A tile's V is read iff some query
+ * head of the group retains it; PV runs only for the retaining heads. The
+ * partial outputs are merged by their log-normalisers:
+ * z = log sum_p exp(z_p), O = sum_p exp(z_p - z) O_p.
+ *
+ * q [B, 1, H_q, d]; k, v [B, N_k, H_kv, d]; o [B, 1, H_q, d]; lse [B, H_q]
+ * fp32; keep_mask optional [B, H_q, ceil(T/32)] uint32.
+ * num_splits: in 0 = let the library choose, else the requested P
+ * (1 <= P <= T); out: the P used (host-side value, known before launch).
+ * Supported: MALA_BF16, d = 128, B_k = 128, H_q / H_kv <= 16.
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  uint32_t* keep_mask;
+  int64_t batch, heads_q, heads_kv, seqlen_k, head_dim;
+  int64_t q_stride[3];
+  int64_t k_stride[3];
+  int64_t v_stride[3];
+  int64_t o_stride[3];
+  const int32_t* q_to_kv;
+  int32_t block_k;
+  float tau;
+  int32_t dtype;
+  int32_t num_splits;
+  int64_t* stats;               /* device int64[4]: tiles tested, V tiles read, head-tiles retained, reserved */
+} mala_decode_args;
+
+MALA_API size_t mala_decode_workspace_size(const mala_decode_args* args);
+MALA_API int mala_decode(mala_decode_args* args, void* workspace, size_t workspace_bytes,
+                void* stream);
+
+/* Human-readable name of a return code. */
+MALA_API const char* mala_status_string(int status);
+
+/* Detail of the last host-side argument error in this thread (never NULL). */
+MALA_API const char* mala_last_error_message(void);
+
+/*
+ * Synchronise `stream` and report a device-side failure recorded by any
+ * kernel of this library since the previous call: MALA_ERR_TIMEOUT if a
+ * bounded wait gave up, MALA_ERR_CUDA if the stream reports a CUDA error,
+ * else MALA_OK. Clears the recorded flag.
+ */
+MALA_API int mala_check_device_error(void* stream);
+
+/* Library version, e.g. "0.1.0". */
+MALA_API const char* mala_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MALA_H_ */

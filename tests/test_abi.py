@@ -1,0 +1,141 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/mala.h declares, the ctypes structs match the C
+layout, and invalid arguments are rejected before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from tile_skipping_causal_b200 import build, mala
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mala.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return mala.load_library()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mala_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared_functions() == sorted(mala.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", mala.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (mala_\w+)", out))
+    for name in _declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+    # nothing else leaks out of the library under the mala_ prefix
+    assert exported == set(_declared_functions())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.mala_version().decode().count(".") == 2
+    for code, name in [(0, "MALA_OK"), (1, "MALA_ERR_INVALID_ARG"), (2, "MALA_ERR_UNSUPPORTED"),
+                       (3, "MALA_ERR_WORKSPACE"), (4, "MALA_ERR_CUDA"), (5, "MALA_ERR_TIMEOUT")]:
+        assert lib.mala_status_string(code).decode() == name
+
+
+def _c_layout(struct, fields):
+    """sizeof/offsetof of a struct in include/mala.h, from a gcc-built probe."""
+    prog = "#include <stdio.h>\n#include <stddef.h>\n#include \"mala.h\"\nint main(void){\n"
+    prog += f'printf("%zu\\n", sizeof({struct}));\n'
+    for f in fields:
+        prog += f'printf("%zu\\n", offsetof({struct}, {f}));\n'
+    prog += "return 0;}\n"
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "probe.c")
+        exe = os.path.join(d, "probe")
+        open(c, "w").write(prog)
+        subprocess.run(["gcc", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True)
+        vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True,
+                                               check=True).stdout.split()]
+    return vals[0], vals[1:]
+
+
+@pytest.mark.parametrize("cls,name", [(mala.FwdArgs, "mala_fwd_args"),
+                                      (mala.BwdArgs, "mala_bwd_args"),
+                                      (mala.DecodeArgs, "mala_decode_args")])
+def test_ctypes_structs_match_c_layout(cls, name):
+    fields = [f[0] for f in cls._fields_]
+    size, offs = _c_layout(name, fields)
+    assert ctypes.sizeof(cls) == size
+    assert [getattr(cls, f).offset for f in fields] == offs
+
+
+def _fwd_args(**kw):
+    a = mala.FwdArgs()
+    fake = 0x10000
+    a.q = a.k = a.v = a.o = a.lse = fake
+    a.batch, a.heads_q, a.heads_kv = 1, 4, 2
+    a.seqlen_q = a.seqlen_k = 256
+    a.head_dim = 128
+    for s in ("q_stride", "o_stride"):
+        setattr(a, s, mala._i64x3(256 * 4 * 128, 4 * 128, 128))
+    for s in ("k_stride", "v_stride"):
+        setattr(a, s, mala._i64x3(256 * 2 * 128, 2 * 128, 128))
+    a.block_q = a.block_k = 128
+    a.tau = 0.1
+    a.dtype = mala.MALA_BF16
+    a.mode = mala.MALA_CAUSAL
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), mala.MALA_ERR_INVALID_ARG),
+    (dict(lse=None), mala.MALA_ERR_INVALID_ARG),
+    (dict(tau=-1.0), mala.MALA_ERR_INVALID_ARG),
+    (dict(tau=float("nan")), mala.MALA_ERR_INVALID_ARG),
+    (dict(heads_kv=3), mala.MALA_ERR_INVALID_ARG),
+    (dict(batch=0), mala.MALA_ERR_INVALID_ARG),
+    (dict(seqlen_q=0, seqlen_k=0), mala.MALA_ERR_INVALID_ARG),
+    (dict(q=0x10008), mala.MALA_ERR_INVALID_ARG),           # misaligned base
+    (dict(q_stride=mala._i64x3(256 * 4 * 128, 4 * 128 + 3, 128)), mala.MALA_ERR_INVALID_ARG),
+    (dict(head_dim=96), mala.MALA_ERR_UNSUPPORTED),
+    (dict(seqlen_k=128), mala.MALA_ERR_UNSUPPORTED),         # causal needs Nq == Nk
+    (dict(block_q=48), mala.MALA_ERR_UNSUPPORTED),
+    (dict(mode=mala.MALA_DECODE), mala.MALA_ERR_UNSUPPORTED),
+    (dict(dtype=7), mala.MALA_ERR_INVALID_ARG),
+])
+def test_fwd_rejects_bad_arguments_without_launching(lib, kw, code):
+    a = _fwd_args(**kw)
+    rc = lib.mala_fwd(ctypes.byref(a), None, 0, None)
+    assert rc == code, lib.mala_last_error_message()
+    assert lib.mala_last_error_message().decode()
+
+
+def test_bad_head_map_rejected(lib):
+    arr = (ctypes.c_int32 * 4)(0, 1, 2, 0)          # 2 is out of range for 2 KV heads
+    a = _fwd_args(q_to_kv=ctypes.cast(arr, ctypes.c_void_p))
+    assert lib.mala_fwd(ctypes.byref(a), None, 0, None) == mala.MALA_ERR_INVALID_ARG
+
+
+def test_null_args_rejected(lib):
+    assert lib.mala_fwd(None, None, 0, None) == mala.MALA_ERR_INVALID_ARG
+    assert lib.mala_bwd(None, None, 0, None) == mala.MALA_ERR_INVALID_ARG
+    assert lib.mala_decode(None, None, 0, None) == mala.MALA_ERR_INVALID_ARG
+
+
+def test_mask_pack_roundtrip():
+    import numpy as np
+    import torch
+    rng = np.random.default_rng(0)
+    m = rng.random((2, 3, 5, 70)) < 0.4
+    w = torch.from_numpy(mala.pack_mask(m))
+    assert w.shape == (2, 3, 5, 3)
+    assert (mala.unpack_mask(w, 70) == m).all()

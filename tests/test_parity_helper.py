@@ -1,0 +1,59 @@
+"""The parity checker accepts correct results and rejects wrong ones (CPU).
+
+Feeds tests/parity.py the oracle's own outputs dressed as GPU tensors, then
+plants mistakes in copies of them (an output element, an LSE entry, a mask
+bit) and checks that each is caught."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import mala_oracle as orc
+from tile_skipping_causal_b200 import mala, synth
+from tests import parity
+
+
+def _case(tau):
+    t = synth.make_prefill(synth.WORKLOADS["prefill_4k"], 3, batch=1, seqlen=300)
+    q, k, v = t["q"], t["k"], t["v"]
+    O, lse, keep, margin = orc.forward(parity.f64(q), parity.f64(k), parity.f64(v), 128, 128, tau)
+    o = torch.from_numpy(O).to(torch.bfloat16)
+    lse_t = torch.from_numpy(lse).float()
+    words = torch.from_numpy(mala.pack_mask(keep))
+    return q, k, v, o, lse_t, words, keep, margin
+
+
+@pytest.mark.parametrize("tau", [0.0, 0.1, 1.0])
+def test_checker_accepts_oracle_output(tau):
+    q, k, v, o, lse, words, keep, _ = _case(tau)
+    rep = parity.check_fwd(q, k, v, o, lse, words, tau, 128, 128)
+    assert rep.blocks == 16 * 3 and rep.replayed_blocks == 0
+
+
+def test_checker_rejects_wrong_output():
+    q, k, v, o, lse, words, keep, _ = _case(0.1)
+    o2 = o.clone()
+    o2[0, 200, 9, 17] += 0.25
+    with pytest.raises(AssertionError, match="O"):
+        parity.check_fwd(q, k, v, o2, lse, words, 0.1, 128, 128)
+    lse2 = lse.clone()
+    lse2[0, 3, 150] += 0.5            # beyond 1e-2 + 2e-2 * |lse|
+    with pytest.raises(AssertionError, match="LSE"):
+        parity.check_fwd(q, k, v, o, lse2, words, 0.1, 128, 128)
+
+
+def test_checker_rejects_wrong_decision():
+    q, k, v, o, lse, words, keep, margin = _case(1.0)
+    # flip a decision far from the threshold: must be reported
+    b, h, i, j = np.argwhere(~np.isnan(margin) & (np.abs(margin) > 0.1) & (np.arange(3)[None, None, :, None] > 0))[0]
+    keep2 = keep.copy()
+    keep2[b, h, i, j] = not keep2[b, h, i, j]
+    with pytest.raises(AssertionError):
+        parity.check_fwd(q, k, v, o, lse, torch.from_numpy(mala.pack_mask(keep2)), 1.0, 128, 128)
+
+
+def test_checker_rejects_bits_above_diagonal():
+    q, k, v, o, lse, words, keep, _ = _case(0.1)
+    keep2 = keep.copy()
+    keep2[0, 0, 0, 2] = True
+    with pytest.raises(AssertionError, match="outside"):
+        parity.check_fwd(q, k, v, o, lse, torch.from_numpy(mala.pack_mask(keep2)), 0.1, 128, 128)

@@ -1,0 +1,53 @@
+// Internal launch interfaces between the C ABI layer (mala_api.cu) and the
+// kernel translation units. Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mala {
+
+constexpr int kMaxHeads = 256;
+
+// Forward, tensor-core path (bf16, B_q = B_k = 128).
+struct FwdTcParams {
+  CUtensorMap tm_q;     // [B, N, Hq, D] as 4-D {D, Hq, N, B}, box {64, 1, 128, 1}, 128B swizzle
+  CUtensorMap tm_k;     // [B, N, Hkv, D]
+  CUtensorMap tm_v;
+  void* o;
+  float* lse;
+  uint32_t* keep_mask;
+  int64_t* stats;
+  int* err;             // library device error word
+  int64_t o_sb, o_sn, o_sh;
+  int B, Hq, Hkv, N;
+  int nQB, nKB, mask_words;
+  float log2_tau;       // log2(tau): -inf for tau = 0, +inf for tau = inf
+  uint8_t kv_of_q[kMaxHeads];
+};
+
+cudaError_t launch_fwd_tc(const FwdTcParams& p, int head_dim, cudaStream_t stream);
+size_t fwd_tc_smem_bytes(int head_dim);
+
+// Forward, CUDA-core path (fp32 or bf16, any supported block sizes).
+struct FwdSimtParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  uint32_t* keep_mask;
+  int64_t* stats;
+  int64_t q_sb, q_sn, q_sh, k_sb, k_sn, k_sh, v_sb, v_sn, v_sh, o_sb, o_sn, o_sh;
+  int B, Hq, Hkv, N;
+  int BQ, BK;
+  int nQB, nKB, mask_words;
+  float log_tau;        // natural log of tau (+-inf allowed)
+  uint8_t kv_of_q[kMaxHeads];
+};
+
+cudaError_t launch_fwd_simt(const FwdSimtParams& p, int head_dim, bool fp32,
+                            cudaStream_t stream);
+
+}  // namespace mala

@@ -1,0 +1,290 @@
+// Host side of the C ABI declared in include/mala.h: argument checks, TMA
+// descriptor encoding, kernel selection and launches. Nothing here allocates
+// device memory; scratch space comes from the caller's workspace.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "kernels.h"
+#include "mala.h"
+
+namespace mala {
+__device__ int g_device_error = 0;
+}  // namespace mala
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MALA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library does not link libcuda directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 4-D bf16 view {d, heads, seq, batch} of a [B, N, H, d] tensor with element
+// strides (sb, sn, sh), box {64, 1, rows, 1}, 128-byte swizzle.
+int make_map_bf16(CUtensorMap* map, const void* ptr, int64_t B, int64_t N, int64_t H, int64_t d,
+                  const int64_t* st, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MALA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)(st[2] * 2), (cuuint64_t)(st[1] * 2), (cuuint64_t)(st[0] * 2)};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MALA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MALA_OK;
+}
+
+// Device address of the error word on the current device.
+int* device_error_ptr() {
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, mala::g_device_error) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks one [B, N, H, d] operand: non-NULL, 16-byte aligned, strides
+// non-negative multiples of 16 bytes, rows that do not overlap.
+int check_tensor(const char* name, const void* p, const int64_t* st, int64_t esize, int64_t d,
+                 int64_t H) {
+  if (!p) return fail(MALA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(MALA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  for (int x = 0; x < 3; ++x) {
+    if (st[x] < 0 || (st[x] * esize) % 16 != 0)
+      return fail(MALA_ERR_INVALID_ARG, "%s stride[%d]=%lld is not a non-negative multiple of 16 bytes",
+                  name, x, (long long)st[x]);
+  }
+  if (st[2] < d) return fail(MALA_ERR_INVALID_ARG, "%s head stride smaller than head_dim", name);
+  if (st[1] < st[2] * H && st[1] != 0)
+    ;  // sequence stride may interleave heads arbitrarily as long as rows are distinct
+  return MALA_OK;
+}
+
+int head_map(const int32_t* q_to_kv, int64_t Hq, int64_t Hkv, uint8_t* out) {
+  if (Hq > mala::kMaxHeads) return fail(MALA_ERR_UNSUPPORTED, "heads_q > %d", mala::kMaxHeads);
+  for (int64_t h = 0; h < Hq; ++h) {
+    int64_t v = q_to_kv ? q_to_kv[h] : h / (Hq / Hkv);
+    if (v < 0 || v >= Hkv) return fail(MALA_ERR_INVALID_ARG, "q_to_kv[%lld]=%lld out of range", (long long)h, (long long)v);
+    out[h] = static_cast<uint8_t>(v);
+  }
+  return MALA_OK;
+}
+
+int check_common(int64_t B, int64_t Hq, int64_t Hkv, int64_t d, float tau, int dtype) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0) return fail(MALA_ERR_INVALID_ARG, "batch and head counts must be positive");
+  if (Hq % Hkv != 0) return fail(MALA_ERR_INVALID_ARG, "heads_q %% heads_kv != 0");
+  if (isnan(tau) || tau < 0.0f) return fail(MALA_ERR_INVALID_ARG, "tau must be >= 0");
+  if (dtype != MALA_BF16 && dtype != MALA_FP32) return fail(MALA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (d != 64 && d != 128) return fail(MALA_ERR_UNSUPPORTED, "head_dim %lld not in {64, 128}", (long long)d);
+  return MALA_OK;
+}
+
+bool block_ok(int x) { return x == 16 || x == 32 || x == 64 || x == 128; }
+
+}  // namespace
+
+extern "C" {
+
+const char* mala_version(void) { return "0.1.0"; }
+
+const char* mala_status_string(int s) {
+  switch (s) {
+    case MALA_OK: return "MALA_OK";
+    case MALA_ERR_INVALID_ARG: return "MALA_ERR_INVALID_ARG";
+    case MALA_ERR_UNSUPPORTED: return "MALA_ERR_UNSUPPORTED";
+    case MALA_ERR_WORKSPACE: return "MALA_ERR_WORKSPACE";
+    case MALA_ERR_CUDA: return "MALA_ERR_CUDA";
+    case MALA_ERR_TIMEOUT: return "MALA_ERR_TIMEOUT";
+    default: return "MALA_ERR_UNKNOWN";
+  }
+}
+
+const char* mala_last_error_message(void) { return g_msg; }
+
+int mala_check_device_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int flag = 0;
+  e = cudaMemcpyFromSymbol(&flag, mala::g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error flag");
+  if (flag != 0) {
+    int zero = 0;
+    cudaMemcpyToSymbol(mala::g_device_error, &zero, sizeof(int));
+    return fail(MALA_ERR_TIMEOUT, "a device-side bounded wait gave up");
+  }
+  return MALA_OK;
+}
+
+// ------------------------------------------------------------------ forward
+
+size_t mala_fwd_workspace_size(const mala_fwd_args* a) {
+  (void)a;
+  return 0;
+}
+
+int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* stream_) {
+  (void)workspace;
+  (void)ws_bytes;
+  g_msg[0] = 0;
+  if (!a) return fail(MALA_ERR_INVALID_ARG, "args is NULL");
+  int rc = check_common(a->batch, a->heads_q, a->heads_kv, a->head_dim, a->tau, a->dtype);
+  if (rc) return rc;
+  if (a->mode != MALA_CAUSAL)
+    return fail(MALA_ERR_UNSUPPORTED, "mala_fwd supports MALA_CAUSAL; use mala_decode for decoding");
+  if (a->seqlen_q <= 0 || a->seqlen_k <= 0) return fail(MALA_ERR_INVALID_ARG, "sequence lengths must be positive");
+  if (a->seqlen_q != a->seqlen_k)
+    return fail(MALA_ERR_UNSUPPORTED, "causal mode needs seqlen_q == seqlen_k");
+  if (a->seqlen_q > (1 << 30)) return fail(MALA_ERR_UNSUPPORTED, "sequence too long");
+  if (!block_ok(a->block_q) || !block_ok(a->block_k))
+    return fail(MALA_ERR_UNSUPPORTED, "block sizes must be in {16, 32, 64, 128}");
+  if (!a->lse) return fail(MALA_ERR_INVALID_ARG, "lse is NULL");
+  const int64_t es = a->dtype == MALA_BF16 ? 2 : 4;
+  const int64_t d = a->head_dim;
+  if ((rc = check_tensor("q", a->q, a->q_stride, es, d, a->heads_q))) return rc;
+  if ((rc = check_tensor("k", a->k, a->k_stride, es, d, a->heads_kv))) return rc;
+  if ((rc = check_tensor("v", a->v, a->v_stride, es, d, a->heads_kv))) return rc;
+  if ((rc = check_tensor("o", a->o, a->o_stride, es, d, a->heads_q))) return rc;
+  if ((reinterpret_cast<uintptr_t>(a->lse) & 3u) != 0) return fail(MALA_ERR_INVALID_ARG, "lse misaligned");
+  if (a->stats && (reinterpret_cast<uintptr_t>(a->stats) & 7u) != 0)
+    return fail(MALA_ERR_INVALID_ARG, "stats misaligned");
+  const int64_t N = a->seqlen_q;
+  const int nQB = static_cast<int>((N + a->block_q - 1) / a->block_q);
+  const int nKB = static_cast<int>((N + a->block_k - 1) / a->block_k);
+  const int mask_words = (nKB + 31) / 32;
+  if ((double)a->batch * a->heads_q * nQB > 2147483647.0) return fail(MALA_ERR_UNSUPPORTED, "grid too large");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+
+  const bool tc = a->dtype == MALA_BF16 && a->block_q == 128 && a->block_k == 128;
+  if (tc) {
+    mala::FwdTcParams p;
+    memset(&p, 0, sizeof(p));
+    if ((rc = head_map(a->q_to_kv, a->heads_q, a->heads_kv, p.kv_of_q))) return rc;
+    if ((rc = make_map_bf16(&p.tm_q, a->q, a->batch, N, a->heads_q, d, a->q_stride, 128))) return rc;
+    if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, N, a->heads_kv, d, a->k_stride, 128))) return rc;
+    if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, N, a->heads_kv, d, a->v_stride, 128))) return rc;
+    p.err = device_error_ptr();
+    if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
+    p.o = a->o;
+    p.lse = a->lse;
+    p.keep_mask = a->keep_mask;
+    p.stats = a->stats;
+    p.o_sb = a->o_stride[0];
+    p.o_sn = a->o_stride[1];
+    p.o_sh = a->o_stride[2];
+    p.B = static_cast<int>(a->batch);
+    p.Hq = static_cast<int>(a->heads_q);
+    p.Hkv = static_cast<int>(a->heads_kv);
+    p.N = static_cast<int>(N);
+    p.nQB = nQB;
+    p.nKB = nKB;
+    p.mask_words = mask_words;
+    p.log2_tau = a->tau == 0.0f ? -INFINITY : log2f(a->tau);
+    cudaError_t e = mala::launch_fwd_tc(p, static_cast<int>(d), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    return MALA_OK;
+  }
+  mala::FwdSimtParams p;
+  memset(&p, 0, sizeof(p));
+  if ((rc = head_map(a->q_to_kv, a->heads_q, a->heads_kv, p.kv_of_q))) return rc;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.o = a->o;
+  p.lse = a->lse;
+  p.keep_mask = a->keep_mask;
+  p.stats = a->stats;
+  p.q_sb = a->q_stride[0]; p.q_sn = a->q_stride[1]; p.q_sh = a->q_stride[2];
+  p.k_sb = a->k_stride[0]; p.k_sn = a->k_stride[1]; p.k_sh = a->k_stride[2];
+  p.v_sb = a->v_stride[0]; p.v_sn = a->v_stride[1]; p.v_sh = a->v_stride[2];
+  p.o_sb = a->o_stride[0]; p.o_sn = a->o_stride[1]; p.o_sh = a->o_stride[2];
+  p.B = static_cast<int>(a->batch);
+  p.Hq = static_cast<int>(a->heads_q);
+  p.Hkv = static_cast<int>(a->heads_kv);
+  p.N = static_cast<int>(N);
+  p.BQ = a->block_q;
+  p.BK = a->block_k;
+  p.nQB = nQB;
+  p.nKB = nKB;
+  p.mask_words = mask_words;
+  p.log_tau = a->tau == 0.0f ? -INFINITY : logf(a->tau);
+  cudaError_t e = mala::launch_fwd_simt(p, static_cast<int>(d), a->dtype == MALA_FP32, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+  return MALA_OK;
+}
+
+// ------------------------------------------------------------------ backward
+
+size_t mala_bwd_workspace_size(const mala_bwd_args* a) {
+  (void)a;
+  return 0;
+}
+
+int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  (void)stream;
+  g_msg[0] = 0;
+  if (!a) return fail(MALA_ERR_INVALID_ARG, "args is NULL");
+  return fail(MALA_ERR_UNSUPPORTED, "backward kernel not built yet");
+}
+
+// ------------------------------------------------------------------ decode
+
+size_t mala_decode_workspace_size(const mala_decode_args* a) {
+  (void)a;
+  return 0;
+}
+
+int mala_decode(mala_decode_args* a, void* workspace, size_t ws_bytes, void* stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  (void)stream;
+  g_msg[0] = 0;
+  if (!a) return fail(MALA_ERR_INVALID_ARG, "args is NULL");
+  return fail(MALA_ERR_UNSUPPORTED, "decode kernel not built yet");
+}
+
+}  // extern "C"
