@@ -114,15 +114,12 @@ def forward_block(Q_i: np.ndarray, pos_i: np.ndarray, K: np.ndarray,
         S = np.where(legal, S, NEG_INF)
         has_key = legal.any(axis=1)          # rows that constrain this tile
 
-        row_margin = np.full(R, math.inf)
-        for q in range(R):
-            if not has_key[q]:
-                continue
-            if l[q] == 0.0:
-                row_margin[q] = NEG_INF      # empty retained set: ratio +inf
-            else:
-                log_ratio = S[q].max() - (m[q] + math.log(l[q]))
-                row_margin[q] = log_thr[q] - log_ratio
+        # per-row slack of the skip test; rows without a legal key do not
+        # constrain (+inf), rows with an empty retained set force retention
+        rmax = np.where(has_key, S.max(axis=1), NEG_INF)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            log_ratio = rmax - (m + np.log(l))
+            row_margin = np.where(has_key, np.where(l > 0.0, log_thr - log_ratio, NEG_INF), math.inf)
         M = float(row_margin.min()) if R else math.inf
         margin[j] = M
         decide = (M <= 0.0)                  # skip iff every row is strictly below
@@ -131,15 +128,14 @@ def forward_block(Q_i: np.ndarray, pos_i: np.ndarray, K: np.ndarray,
         keep[j] = decide
 
         if decide:
-            for q in range(R):
-                if not has_key[q]:
-                    continue
-                m_new = max(m[q], S[q].max())
-                p = np.exp(S[q] - m_new)     # exp(-inf) = 0 on illegal keys
-                alpha = math.exp(m[q] - m_new) if l[q] > 0.0 else 0.0
-                l[q] = l[q] * alpha + p.sum()
-                acc[q] = acc[q] * alpha + p @ V[k0:k1]
-                m[q] = m_new
+            # standard online-softmax update of the rows with a legal key
+            rows = np.nonzero(has_key)[0]
+            m_new = np.maximum(m[rows], rmax[rows])
+            p = np.exp(S[rows] - m_new[:, None])            # exp(-inf) = 0 on illegal keys
+            alpha = np.where(l[rows] > 0.0, np.exp(m[rows] - m_new), 0.0)
+            l[rows] = l[rows] * alpha + p.sum(axis=1)
+            acc[rows] = acc[rows] * alpha[:, None] + p @ V[k0:k1]
+            m[rows] = m_new
         if trace is not None:
             trace(j, dict(m=m.copy(), l=l.copy(), keep=decide, S=S, margin=M))
 
