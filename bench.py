@@ -128,7 +128,7 @@ def run_mala(args):
     mala.load_library()
 
     w = synth.WORKLOADS[WORKLOAD]
-    t = synth.make_prefill(w, SEED + rank, with_do=True)
+    t = synth.make_prefill(w, SEED + rank, with_do=True, seqlen=args.seqlen)
     host = {n: x.pin_memory() for n, x in t.items()}
     q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
     B, N, Hq, d = q.shape
@@ -181,6 +181,13 @@ def run_mala(args):
     ms_per_step = elapsed / args.steps * 1e3
     tokens = B * N * world * args.steps
     value = tokens / elapsed
+
+    if args.no_extras:
+        if rank == 0:
+            print(json.dumps({"profile_case": True, "seqlen": N, "ms_per_step": ms_per_step}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     # dense comparison: the same kernels at tau = 0
     stats.zero_()
@@ -330,11 +337,15 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["mala", "reference"], default="mala")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="shrink N (same recipe); for profiling captures only")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time the step only (no tau=0, e2e, baseline); for profiling captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

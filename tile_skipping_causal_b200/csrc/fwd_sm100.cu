@@ -95,7 +95,9 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
   uint8_t* sP = smem + L::kP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L::kMisc);
-  // misc[0] TMEM base, misc[1] abort flag, misc[2..3] decisions of tiles t&1
+  // misc[0] TMEM base, misc[1] abort flag, misc[2..4] progress markers of the
+  // producer / MMA / softmax roles (kept for timeout diagnosis), misc[5..6]
+  // decisions of tiles t & 1
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
   const int tid = threadIdx.x;
@@ -122,6 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       mbar_init(&bars[x], cnt);
     }
     misc[1] = 0;
+    misc[2] = misc[3] = misc[4] = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -143,13 +146,15 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       mbar_expect_tx(&bars[kQFull], L::kTile);
       for (int c = 0; c < NCH; ++c)
         tma_load_4d(sQ + c * kChunkBytes, &p.tm_q, &bars[kQFull], c * 64, h, q0, b);
+      misc[2] = 0x10000u;
       auto load_k = [&](int t) -> bool {
         const int s = t & 1;
-        if (!mbar_wait(&bars[kKEmpty + s], ((t >> 1) & 1) ^ 1, abort_flag, p.err)) return false;
+        if (!mbar_wait(&bars[kKEmpty + s], ((t >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(1, kKEmpty + s, t))) return false;
         mbar_expect_tx(&bars[kKFull + s], L::kTile);
         for (int c = 0; c < NCH; ++c)
           tma_load_4d(sK + s * L::kTile + c * kChunkBytes, &p.tm_k, &bars[kKFull + s], c * 64, hk,
                       (j_diag - t) * kBK, b);
+        misc[2] = 0x20000u | t;
         return true;
       };
       bool ok = load_k(0);
@@ -157,12 +162,13 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       int kc = 0;
       for (int t = 0; ok && t < T; ++t) {
         const int s = t & 1;
-        if (!mbar_wait(&bars[kDecFull + s], (t >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
-        const uint32_t keep = misc[2 + s];
+        if (!mbar_wait(&bars[kDecFull + s], (t >> 1) & 1, abort_flag, p.err, wait_tag(1, kDecFull + s, t))) { ok = false; break; }
+        const uint32_t keep = misc[5 + s];
         mbar_arrive(&bars[kDecEmpty + s]);
+        misc[2] = 0x30000u | t;
         if (keep) {
           const int vs = kc & 1;
-          if (!mbar_wait(&bars[kVEmpty + vs], ((kc >> 1) & 1) ^ 1, abort_flag, p.err)) { ok = false; break; }
+          if (!mbar_wait(&bars[kVEmpty + vs], ((kc >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(1, kVEmpty + vs, kc))) { ok = false; break; }
           mbar_expect_tx(&bars[kVFull + vs], L::kTile);
           for (int c = 0; c < NCH; ++c)
             tma_load_4d(sV + vs * L::kTile + c * kChunkBytes, &p.tm_v, &bars[kVFull + vs], c * 64,
@@ -181,8 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
       auto issue_qk = [&](int t) -> bool {
         const int s = t & 1;
-        if (!mbar_wait(&bars[kKFull + s], (t >> 1) & 1, abort_flag, p.err)) return false;
-        if (!mbar_wait(&bars[kSEmpty + s], ((t >> 1) & 1) ^ 1, abort_flag, p.err)) return false;
+        if (!mbar_wait(&bars[kKFull + s], (t >> 1) & 1, abort_flag, p.err, wait_tag(2, kKFull + s, t))) return false;
+        if (!mbar_wait(&bars[kSEmpty + s], ((t >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(2, kSEmpty + s, t))) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
@@ -193,22 +199,24 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
         }
         umma_commit(&bars[kSFull + s]);
         umma_commit(&bars[kKEmpty + s]);
+        misc[3] = 0x20000u | t;
         return true;
       };
-      bool ok = mbar_wait(&bars[kQFull], 0, abort_flag, p.err);
+      bool ok = mbar_wait(&bars[kQFull], 0, abort_flag, p.err, wait_tag(2, kQFull, 0));
+      if (ok) misc[3] = 0x10000u;
       if (ok) ok = issue_qk(0);
       if (ok && T > 1) ok = issue_qk(1);
       int kc = 0;
       for (int t = 0; ok && t < T; ++t) {
         const int s = t & 1;
-        if (!mbar_wait(&bars[kDecFull + s], (t >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
-        const uint32_t keep = misc[2 + s];
+        if (!mbar_wait(&bars[kDecFull + s], (t >> 1) & 1, abort_flag, p.err, wait_tag(2, kDecFull + s, t))) { ok = false; break; }
+        const uint32_t keep = misc[5 + s];
         mbar_arrive(&bars[kDecEmpty + s]);
         if (t + 2 < T && !issue_qk(t + 2)) { ok = false; break; }
         if (keep) {
           const int ps = kc & 1;
-          if (!mbar_wait(&bars[kPFull + ps], (kc >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
-          if (!mbar_wait(&bars[kVFull + ps], (kc >> 1) & 1, abort_flag, p.err)) { ok = false; break; }
+          if (!mbar_wait(&bars[kPFull + ps], (kc >> 1) & 1, abort_flag, p.err, wait_tag(2, kPFull + ps, kc))) { ok = false; break; }
+          if (!mbar_wait(&bars[kVFull + ps], (kc >> 1) & 1, abort_flag, p.err, wait_tag(2, kVFull + ps, kc))) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
@@ -219,12 +227,13 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
           }
           umma_commit(&bars[kPEmpty + ps]);
           umma_commit(&bars[kVEmpty + ps]);
+          misc[3] = 0x40000u | t;
           ++kc;
         }
       }
       // make sure every MMA issued above has finished before TMEM is freed
       umma_commit(&bars[kMmaDone]);
-      mbar_wait(&bars[kMmaDone], 0, abort_flag, p.err);
+      mbar_wait(&bars[kMmaDone], 0, abort_flag, p.err, wait_tag(2, kMmaDone, 0));
     }
   } else {
     // ===================== softmax warpgroup =====================
@@ -249,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       const int s = t & 1;
       uint32_t sr[4][32];
       // tcgen05.ld is warp-collective: load only if every lane's wait succeeded
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull + s], (t >> 1) & 1, abort_flag, p.err));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull + s], (t >> 1) & 1, abort_flag, p.err, wait_tag(0, kSFull + s, t)));
       if (ok) {
         tc_fence_after();
 #pragma unroll
@@ -267,6 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
       tc_fence_before();
       mbar_arrive(&bars[kSEmpty + s]);
+      if (tid == 0) misc[4] = (ok ? 0x10000u : 0x90000u) | t;
 
       // causal mask: key k = j*128 + c is legal iff k <= q
       const int lim = q - j * kBK;           // largest legal column index
@@ -285,12 +295,14 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       // an empty retained set (l = 0) always retains
       const bool vote = has_key && (l == 0.0f || rmax2 - (m2 + lg2_approx(l)) >= thr2);
       const bool keep = bar_or(1, kBQ, vote);
-      if (*abort_flag, p.err) break;
+      if (tid == 0) misc[4] = 0x20000u | t;
+      if (*abort_flag) break;
 
       if (tid == 0) {
-        if (mbar_wait(&bars[kDecEmpty + s], ((t >> 1) & 1) ^ 1, abort_flag, p.err)) {
-          misc[2 + s] = keep ? 1u : 0u;
+        if (mbar_wait(&bars[kDecEmpty + s], ((t >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty + s, t))) {
+          misc[5 + s] = keep ? 1u : 0u;
           mbar_arrive(&bars[kDecFull + s]);
+          misc[4] = 0x30000u | t;
         }
         if (keep) {
           mask_word |= 1u << (j & 31);
@@ -320,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       if (kc > 0 && __any_sync(0xffffffffu, rescale)) {
         {
           // O holds PV of earlier retained tiles: wait for the last one
-          mbar_wait(&bars[kPEmpty + ((kc - 1) & 1)], ((kc - 1) >> 1) & 1, abort_flag, p.err);
+          mbar_wait(&bars[kPEmpty + ((kc - 1) & 1)], ((kc - 1) >> 1) & 1, abort_flag, p.err, wait_tag(0, kPEmpty + ((kc - 1) & 1), kc));
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -338,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       m2 = new_m2;
 
       // P buffer kc & 1 is free once PV(kc - 2) has completed
-      mbar_wait(&bars[kPEmpty + (kc & 1)], ((kc >> 1) & 1) ^ 1, abort_flag, p.err);
+      mbar_wait(&bars[kPEmpty + (kc & 1)], ((kc >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(0, kPEmpty + (kc & 1), kc));
       const float neg_m2 = has_key ? -m2 : 0.0f;
       float psum = 0.0f;
       const uint32_t prow = sPa + (kc & 1) * kPBytes + r * 128;
@@ -369,8 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
     }
 
     // ---- epilogue: O = acc / l (bf16), z = (m2 + log2 l) ln 2, mask, stats
-    if (!*abort_flag, p.err) {
-      if (kc > 0) mbar_wait(&bars[kPEmpty + ((kc - 1) & 1)], ((kc - 1) >> 1) & 1, abort_flag, p.err);
+    if (!*abort_flag) {
+      if (kc > 0) mbar_wait(&bars[kPEmpty + ((kc - 1) & 1)], ((kc - 1) >> 1) & 1, abort_flag, p.err, wait_tag(0, kPEmpty + ((kc - 1) & 1), kc));
       tc_fence_after();
       const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + b * p.o_sb +

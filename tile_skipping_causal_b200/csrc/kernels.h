@@ -19,7 +19,7 @@ struct FwdTcParams {
   float* lse;
   uint32_t* keep_mask;
   int64_t* stats;
-  int* err;             // library device error word
+  int* err;             // library device error block int[4]
   int64_t o_sb, o_sn, o_sh;
   int B, Hq, Hkv, N;
   int nQB, nKB, mask_words;

@@ -14,7 +14,9 @@
 #include "mala.h"
 
 namespace mala {
-__device__ int g_device_error = 0;
+// {code, tag, block, parity, progress x3, spare} of the first device-side
+// wait that gave up
+__device__ int g_device_error[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 }  // namespace mala
 
 namespace {
@@ -71,7 +73,7 @@ int make_map_bf16(CUtensorMap* map, const void* ptr, int64_t B, int64_t N, int64
   return MALA_OK;
 }
 
-// Device address of the error word on the current device.
+// Device address of the error block on the current device.
 int* device_error_ptr() {
   static int* ptrs[64] = {nullptr};
   int dev = 0;
@@ -147,13 +149,17 @@ const char* mala_last_error_message(void) { return g_msg; }
 int mala_check_device_error(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
-  int flag = 0;
-  e = cudaMemcpyFromSymbol(&flag, mala::g_device_error, sizeof(int));
+  int rec[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  e = cudaMemcpyFromSymbol(rec, mala::g_device_error, sizeof(rec));
   if (e != cudaSuccess) return cuda_fail(e, "read device error flag");
-  if (flag != 0) {
-    int zero = 0;
-    cudaMemcpyToSymbol(mala::g_device_error, &zero, sizeof(int));
-    return fail(MALA_ERR_TIMEOUT, "a device-side bounded wait gave up");
+  if (rec[0] != 0) {
+    int zero[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    cudaMemcpyToSymbol(mala::g_device_error, zero, sizeof(zero));
+    return fail(MALA_ERR_TIMEOUT,
+                "a device-side bounded wait gave up (role %d, barrier %d, tile %d, block %d, parity %d; "
+                "progress %08x %08x %08x)",
+                (rec[1] >> 24) & 0xf, (rec[1] >> 16) & 0xff, rec[1] & 0xffff, rec[2], rec[3], rec[4],
+                rec[5], rec[6]);
   }
   return MALA_OK;
 }

@@ -67,9 +67,12 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 
 // Wait for the phase of `bar` with parity `parity` to complete. Gives up
 // when *abort becomes non-zero (another thread gave up) or after
-// kWaitLimitNs; then sets *abort, records the timeout and returns false.
+// kWaitLimitNs; then sets *abort and records the timeout in the error block
+// err[0..6] = {code, tag of the first wait that gave up, its block index,
+// its parity, progress words abort[1..3]}. `tag` identifies the wait site
+// (role, barrier, tile); abort[1..3] must be readable shared words.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort, int* err) {
+                                          volatile int* abort, int* err, int tag = 0) {
   if (mbar_test(bar, parity)) return true;
   uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -78,11 +81,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
       if (*abort) return false;
       if (global_timer_ns() - t0 > kWaitLimitNs) {
         *abort = 1;
-        atomicExch(err, kErrTimeout);
+        if (atomicCAS(err, 0, kErrTimeout) == 0) {
+          err[1] = tag;
+          err[2] = static_cast<int>(blockIdx.x);
+          err[3] = static_cast<int>(parity);
+          // the three words after the abort flag hold the CTA's per-role
+          // progress markers (see the kernels); keep them for diagnosis
+          for (int x = 0; x < 3; ++x) err[4 + x] = abort[1 + x];
+        }
         return false;
       }
     }
   }
+}
+
+// Tag of a wait site: role (4 bits), barrier index (8 bits), tile (16 bits).
+__host__ __device__ constexpr int wait_tag(int role, int bar, int tile) {
+  return (role << 24) | ((bar & 0xff) << 16) | (tile & 0xffff);
 }
 
 // Bounded pause used on the abort path so that copies already in flight
