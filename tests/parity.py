@@ -113,3 +113,56 @@ def check_fwd(q, k, v, o, lse, keep_words, tau, B_q, B_k, samples=None, rep=None
             check_fwd_block(Qh[q0:q1], Kh, Vh, pos, tiles, B_k, tau, keep[b, h, i], Oh[q0:q1],
                             lse_c[b, h, q0:q1], rep, f"fwd b={b} h={h} i={i}")
     return rep
+
+
+class DecReport:
+    def __init__(self):
+        self.heads = 0
+        self.tiles = 0
+        self.kept = 0
+        self.band_flips = 0
+        self.replayed = 0
+
+
+def check_decode_head(q_row, K, V, B_k, tau, P, gpu_keep_row, gpu_o, gpu_lse, rep, what):
+    """One (batch, query head) of mala_decode against the oracle's split-KV
+    decode with the same split count."""
+    O, z, keep, margin, _ = orc.decode_head(q_row, K, V, B_k, tau, P)
+    nKB = len(keep)
+    gk = np.asarray(gpu_keep_row[:nKB], dtype=bool)
+    if (keep != gk).any():
+        rep.replayed += 1
+        O, z, keep, margin, _ = orc.decode_head(q_row, K, V, B_k, tau, P, replay=gk)
+    for j in range(nKB):
+        if gk[j] != (margin[j] <= 0.0):
+            assert abs(margin[j]) <= MARGIN_BAND, f"{what}: tile {j} decided {gk[j]} with margin {margin[j]:.3e}"
+            rep.band_flips += 1
+    assert_close(gpu_o, O, f"{what} O")
+    assert_close(np.array([gpu_lse]), np.array([z]), f"{what} LSE")
+    rep.heads += 1
+    rep.tiles += nKB
+    rep.kept += int(gk.sum())
+
+
+def check_decode(q, k, v, o, lse, keep_words, tau, P, B_k=128, heads=None, rep=None):
+    """mala_decode outputs vs the oracle for (b, h) pairs ``heads`` (None = all).
+    q [B, 1, Hq, d]; k/v [B, Nk, Hkv, d] (device or host tensors)."""
+    rep = rep or DecReport()
+    B, _, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    nKB = orc.num_blocks(Nk, B_k)
+    keep = mala.unpack_mask(keep_words, nKB)
+    if heads is None:
+        heads = [(b, h) for b in range(B) for h in range(Hq)]
+    o_c = f64(o)
+    lse_c = lse.detach().cpu().numpy()
+    by_kv = {}
+    for (b, h) in heads:
+        by_kv.setdefault((b, h // G), []).append(h)
+    for (b, hk), hs in by_kv.items():
+        K, V = f64(k[b, :, hk]), f64(v[b, :, hk])
+        for h in hs:
+            check_decode_head(f64(q[b, 0, h]), K, V, B_k, tau, P, keep[b, h], o_c[b, 0, h],
+                              float(lse_c[b, h]), rep, f"decode b={b} h={h}")
+    return rep

@@ -1,0 +1,115 @@
+"""GPU parity of mala_decode (split-KV decoding) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import mala_oracle as orc
+from tile_skipping_causal_b200 import mala, synth
+from tests.parity import check_decode
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+SEED = 42
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from tile_skipping_causal_b200 import build
+    build.build()
+    mala.load_library()
+
+
+def _decode(q, k, v, tau, splits=0, **kw):
+    o, lse, keep, P = mala.mala_decode(q, k, v, tau, 128, splits, **kw)
+    mala.check_device_error()
+    return o, lse, keep, P
+
+
+def _small(batch, Nk, seed=SEED, Hq=32, Hkv=8):
+    w = synth.DecodeWorkload("decode_small", batch, Hq, Hkv, Nk, 128, 128, 0.05)
+    q = synth.make_decode_query(w, seed)
+    k, v = synth.fill_decode_cache(w, seed, q, DEV)
+    return w, q.to(DEV), k, v
+
+
+@pytest.mark.parametrize("Nk", [300, 1000, 4096])
+@pytest.mark.parametrize("splits", [1, 3, 0])
+def test_decode_recipe_reduced_all_heads(Nk, splits):
+    w, q, k, v = _small(2, Nk)
+    o, lse, keep, P = _decode(q, k, v, w.tau, splits)
+    if splits:
+        assert P == splits
+    rep = check_decode(q, k, v, o, lse, keep, w.tau, P)
+    assert rep.heads == 2 * 32
+
+
+@pytest.mark.parametrize("Nk", synth.DECODE_SEQLENS)
+def test_decode_full_size_sampled(Nk):
+    w = synth.decode_workload(Nk)
+    q = synth.make_decode_query(w, SEED)
+    sample_kv = [(0, 0), (17, 3), (63, 7)]
+    k, v = synth.fill_decode_cache(w, SEED, q, DEV, slices=sample_kv)
+    qd = q.to(DEV)
+    o, lse, keep, P = _decode(qd, k, v, w.tau)
+    heads = [(b, hk * 4 + g) for (b, hk) in sample_kv for g in range(4)]
+    rep = check_decode(qd, k, v, o, lse, keep, w.tau, P, heads=heads)
+    assert rep.heads == len(heads)
+    del k, v
+    torch.cuda.empty_cache()
+
+
+def test_decode_tau_zero_is_dense():
+    w, q, k, v = _small(1, 777)
+    o, lse, keep, P = _decode(q, k, v, 0.0, 2)
+    assert mala.unpack_mask(keep, 7).all()
+    check_decode(q, k, v, o, lse, keep, 0.0, P)
+
+
+def test_decode_tau_inf_keeps_first_tile_of_each_split():
+    w, q, k, v = _small(1, 1280)
+    o, lse, keep, P = _decode(q, k, v, math.inf, 3)
+    m = mala.unpack_mask(keep, 10)
+    expect = np.zeros(10, dtype=bool)
+    for (t0, t1) in orc.split_ranges(10, 3):
+        expect[t1 - 1] = True
+    assert (m == expect[None, None]).all()
+    check_decode(q, k, v, o, lse, keep, math.inf, P)
+
+
+@pytest.mark.parametrize("Nk", [1, 127, 128, 129])
+def test_decode_edge_lengths(Nk):
+    w, q, k, v = _small(2, Nk)
+    o, lse, keep, P = _decode(q, k, v, 0.05)
+    check_decode(q, k, v, o, lse, keep, 0.05, P)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 1), (6, 2)])
+def test_decode_group_sizes(Hq, Hkv):
+    w, q, k, v = _small(2, 640, Hq=Hq, Hkv=Hkv)
+    o, lse, keep, P = _decode(q, k, v, 0.05, 2)
+    check_decode(q, k, v, o, lse, keep, 0.05, P)
+
+
+def test_decode_explicit_head_map():
+    w, q, k, v = _small(1, 512, Hq=4, Hkv=2)
+    hmap = [1, 0, 0, 1]
+    o, lse, keep, P = _decode(q, k, v, 0.05, 2, q_to_kv=hmap)
+    kp = k[:, :, hmap].contiguous()
+    vp = v[:, :, hmap].contiguous()
+    # the oracle reads the same map through per-head copies (group of 1)
+    check_decode(q, kp, vp, o, lse, keep, 0.05, P)
+
+
+def test_decode_stats():
+    w, q, k, v = _small(1, 2048)
+    stats = torch.zeros(4, dtype=torch.int64, device=DEV)
+    o, lse, keep, P = _decode(q, k, v, 0.05, 4, stats=stats)
+    m = mala.unpack_mask(keep, 16)
+    s = stats.cpu().tolist()
+    assert s[0] == 8 * 16                     # (b, kv head) x tiles
+    assert s[2] == m.sum()                    # head-tiles retained
+    grp = m.reshape(1, 8, 4, 16).any(axis=2)  # V read iff some head of the group retains
+    assert s[1] == grp.sum()

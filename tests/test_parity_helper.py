@@ -57,3 +57,30 @@ def test_checker_rejects_bits_above_diagonal():
     keep2[0, 0, 0, 2] = True
     with pytest.raises(AssertionError, match="outside"):
         parity.check_fwd(q, k, v, o, lse, torch.from_numpy(mala.pack_mask(keep2)), 0.1, 128, 128)
+
+
+def _dec_case(tau, P):
+    w = synth.DecodeWorkload("d", 1, 8, 2, 700, 128, 128, tau)
+    q = synth.make_decode_query(w, 5)
+    k, v = synth.fill_decode_cache(w, 5, q, "cpu")
+    O, lse, keep, margin = orc.decode(parity.f64(q), parity.f64(k), parity.f64(v), 128, tau, P)
+    return q, k, v, torch.from_numpy(O).to(torch.bfloat16), torch.from_numpy(lse).float(), keep, margin
+
+
+def test_decode_checker_accepts_oracle_output():
+    q, k, v, o, lse, keep, _ = _dec_case(0.05, 2)
+    rep = parity.check_decode(q, k, v, o, lse, torch.from_numpy(mala.pack_mask(keep)), 0.05, 2)
+    assert rep.heads == 8 and rep.replayed == 0
+
+
+def test_decode_checker_rejects_wrong_decision_and_output():
+    q, k, v, o, lse, keep, margin = _dec_case(2.0, 1)
+    b, h, j = np.argwhere(~np.isnan(margin) & (np.abs(margin) > 0.1))[0]
+    keep2 = keep.copy()
+    keep2[b, h, j] = not keep2[b, h, j]
+    with pytest.raises(AssertionError):
+        parity.check_decode(q, k, v, o, lse, torch.from_numpy(mala.pack_mask(keep2)), 2.0, 1)
+    o2 = o.clone()
+    o2[0, 0, 3, 5] += 0.3
+    with pytest.raises(AssertionError, match="O"):
+        parity.check_decode(q, k, v, o2, lse, torch.from_numpy(mala.pack_mask(keep)), 2.0, 1)

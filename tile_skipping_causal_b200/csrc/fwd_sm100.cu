@@ -296,7 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       const bool vote = has_key && (l == 0.0f || rmax2 - (m2 + lg2_approx(l)) >= thr2);
       const bool keep = bar_or(1, kBQ, vote);
       if (tid == 0) misc[4] = 0x20000u | t;
-      if (*abort_flag) break;
+      // every softmax thread must leave at the same tile: OR the flag through a barrier
+      if (bar_or(1, kBQ, *abort_flag != 0)) break;
 
       if (tid == 0) {
         if (mbar_wait(&bars[kDecEmpty + s], ((t >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty + s, t))) {

@@ -50,4 +50,29 @@ struct FwdSimtParams {
 cudaError_t launch_fwd_simt(const FwdSimtParams& p, int head_dim, bool fp32,
                             cudaStream_t stream);
 
+// Split-KV decoding (bf16, d = 128, B_k = 128, group size <= 16).
+constexpr int kMaxKvHeads = 64;
+constexpr int kMaxGroup = 16;
+
+struct DecodeParams {
+  CUtensorMap tm_k;     // [B, Nk, Hkv, 128] as 4-D, box {64, 1, 128, 1}, 128B swizzle
+  CUtensorMap tm_v;
+  const void* q;        // [B, 1, Hq, 128]
+  void* o;              // [B, 1, Hq, 128]
+  float* lse;           // [B, Hq]
+  uint32_t* keep_mask;  // [B, Hq, mask_words] (zeroed by the host before the launch)
+  int64_t* stats;
+  int* err;
+  float* part_o;        // [B, Hq, P, 128] fp32 (P > 1)
+  float* part_lse;      // [B, Hq, P]
+  int64_t q_sb, q_sh, o_sb, o_sh;
+  int B, Hq, Hkv, Nk, nKB, mask_words, num_splits;
+  float log2_tau;
+  uint8_t group_size[kMaxKvHeads];
+  uint8_t group_heads[kMaxKvHeads][kMaxGroup];
+};
+
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
+size_t decode_smem_bytes();
+
 }  // namespace mala

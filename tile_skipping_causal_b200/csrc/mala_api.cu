@@ -279,18 +279,117 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
 
 // ------------------------------------------------------------------ decode
 
-size_t mala_decode_workspace_size(const mala_decode_args* a) {
-  (void)a;
-  return 0;
+namespace {
+
+int decode_check(const mala_decode_args* a, int* nKB_out) {
+  int rc = check_common(a->batch, a->heads_q, a->heads_kv, a->head_dim, a->tau, a->dtype);
+  if (rc) return rc;
+  if (a->dtype != MALA_BF16) return fail(MALA_ERR_UNSUPPORTED, "decode supports bf16 only");
+  if (a->head_dim != 128) return fail(MALA_ERR_UNSUPPORTED, "decode supports head_dim 128 only");
+  if (a->block_k != 128) return fail(MALA_ERR_UNSUPPORTED, "decode supports block_k 128 only");
+  if (a->seqlen_k <= 0) return fail(MALA_ERR_INVALID_ARG, "seqlen_k must be positive");
+  if (a->seqlen_k > (1 << 30)) return fail(MALA_ERR_UNSUPPORTED, "cache too long");
+  if (a->heads_kv > mala::kMaxKvHeads) return fail(MALA_ERR_UNSUPPORTED, "heads_kv > %d", mala::kMaxKvHeads);
+  if (!a->lse) return fail(MALA_ERR_INVALID_ARG, "lse is NULL");
+  const int nKB = static_cast<int>((a->seqlen_k + 127) / 128);
+  if (a->num_splits < 0 || a->num_splits > nKB)
+    return fail(MALA_ERR_INVALID_ARG, "num_splits %d outside [0, %d]", a->num_splits, nKB);
+  if ((rc = check_tensor("q", a->q, a->q_stride, 2, 128, a->heads_q))) return rc;
+  if ((rc = check_tensor("k", a->k, a->k_stride, 2, 128, a->heads_kv))) return rc;
+  if ((rc = check_tensor("v", a->v, a->v_stride, 2, 128, a->heads_kv))) return rc;
+  if ((rc = check_tensor("o", a->o, a->o_stride, 2, 128, a->heads_q))) return rc;
+  *nKB_out = nKB;
+  return MALA_OK;
 }
 
-int mala_decode(mala_decode_args* a, void* workspace, size_t ws_bytes, void* stream) {
-  (void)workspace;
-  (void)ws_bytes;
-  (void)stream;
+// Splits per (batch, KV head): enough CTAs for several waves over the SMs,
+// at least 4 key tiles per split.
+int choose_splits(int64_t units, int nKB) {
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) sms = v;
+  }
+  int64_t want = (8LL * sms + units - 1) / units;
+  int64_t cap = nKB / 4 > 0 ? nKB / 4 : 1;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  return static_cast<int>(want);
+}
+
+size_t decode_ws_bytes(const mala_decode_args* a, int P) {
+  if (P <= 1) return 0;
+  return static_cast<size_t>(a->batch) * a->heads_q * P * (128 + 1) * sizeof(float) + 256;
+}
+
+}  // namespace
+
+size_t mala_decode_workspace_size(const mala_decode_args* a) {
+  if (!a) return 0;
+  int nKB = 0;
+  if (decode_check(a, &nKB) != MALA_OK) return 0;
+  const int P = a->num_splits > 0 ? a->num_splits : choose_splits(a->batch * a->heads_kv, nKB);
+  return decode_ws_bytes(a, P);
+}
+
+int mala_decode(mala_decode_args* a, void* workspace, size_t ws_bytes, void* stream_) {
   g_msg[0] = 0;
   if (!a) return fail(MALA_ERR_INVALID_ARG, "args is NULL");
-  return fail(MALA_ERR_UNSUPPORTED, "decode kernel not built yet");
+  int nKB = 0;
+  int rc = decode_check(a, &nKB);
+  if (rc) return rc;
+  const int P = a->num_splits > 0 ? a->num_splits : choose_splits(a->batch * a->heads_kv, nKB);
+  const size_t need = decode_ws_bytes(a, P);
+  if (need > 0 && (!workspace || ws_bytes < need))
+    return fail(MALA_ERR_WORKSPACE, "decode workspace of %zu bytes needed", need);
+  if (need > 0 && !aligned16(workspace)) return fail(MALA_ERR_INVALID_ARG, "workspace misaligned");
+
+  mala::DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  uint8_t kv_of_q[mala::kMaxHeads];
+  if ((rc = head_map(a->q_to_kv, a->heads_q, a->heads_kv, kv_of_q))) return rc;
+  for (int64_t h = 0; h < a->heads_q; ++h) {
+    const int hk = kv_of_q[h];
+    if (p.group_size[hk] >= mala::kMaxGroup)
+      return fail(MALA_ERR_UNSUPPORTED, "more than %d query heads share KV head %d", mala::kMaxGroup, hk);
+    p.group_heads[hk][p.group_size[hk]++] = static_cast<uint8_t>(h);
+  }
+  if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, a->seqlen_k, a->heads_kv, 128, a->k_stride, 128))) return rc;
+  if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, a->seqlen_k, a->heads_kv, 128, a->v_stride, 128))) return rc;
+  p.err = device_error_ptr();
+  if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
+  p.q = a->q;
+  p.o = a->o;
+  p.lse = a->lse;
+  p.keep_mask = a->keep_mask;
+  p.stats = a->stats;
+  if (P > 1) {
+    p.part_o = static_cast<float*>(workspace);
+    p.part_lse = p.part_o + static_cast<size_t>(a->batch) * a->heads_q * P * 128;
+  }
+  p.q_sb = a->q_stride[0];
+  p.q_sh = a->q_stride[2];
+  p.o_sb = a->o_stride[0];
+  p.o_sh = a->o_stride[2];
+  p.B = static_cast<int>(a->batch);
+  p.Hq = static_cast<int>(a->heads_q);
+  p.Hkv = static_cast<int>(a->heads_kv);
+  p.Nk = static_cast<int>(a->seqlen_k);
+  p.nKB = nKB;
+  p.mask_words = (nKB + 31) / 32;
+  p.num_splits = P;
+  p.log2_tau = a->tau == 0.0f ? -INFINITY : log2f(a->tau);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (a->keep_mask) {
+    cudaError_t e = cudaMemsetAsync(a->keep_mask, 0,
+                                    static_cast<size_t>(a->batch) * a->heads_q * p.mask_words * 4, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "keep mask clear");
+  }
+  cudaError_t e = mala::launch_decode(p, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  a->num_splits = P;
+  return MALA_OK;
 }
 
 }  // extern "C"

@@ -298,3 +298,44 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 }
 
 }  // namespace mala
+
+namespace mala {
+
+// ------------------------------------------------------------------ warp MMA (mma.sync)
+
+// Four 8x8 b16 matrices from shared memory; lane l supplies the row address
+// of matrix l / 8, row l % 8.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte address of the 16-byte unit holding elements [d0, d0 + 8) of row
+// `row` in a TMA tile loaded with 128-byte swizzle as 64-element chunks of
+// 128 rows (chunk c at c * 16 KB, row r at r * 128 B, unit u at u ^ (r & 7)).
+__device__ __forceinline__ uint32_t sw128_addr(uint32_t base, int row, int d0) {
+  const int c = d0 >> 6;
+  const int u = (d0 & 63) >> 3;
+  return base + c * 16384 + row * 128 + ((u ^ (row & 7)) << 4);
+}
+
+}  // namespace mala
