@@ -5,8 +5,8 @@
 Workload (per GPU): long-context GQA prefill, batch 1, 32 query heads, 8 KV
 heads, N = 32768, d = 128, 128 x 128 tiles, bf16, causal, heads in thirds
 (diffuse / local / retrieval), tau = 0.2. One step = one pass of the hot path
-over that batch: the MALA forward, then (when built) the MALA backward with
-dO ~ N(0, 1). Inputs (~0.4 GB) are larger than the 126 MB L2.
+over that batch: the MALA forward, then the MALA backward (mask replay)
+with dO ~ N(0, 1). Inputs (~0.7 GB) are larger than the 126 MB L2.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own batch
 (independent problems, no data-path collective), time = max over ranks,
@@ -138,26 +138,41 @@ def run_mala(args):
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
     keep = torch.empty((B, Hq, nQB, mala.mask_words(nKB)), dtype=torch.int32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     stats = torch.zeros(4, dtype=torch.int64, device=dev)
-    launches_per_step = 1
+    bstats = torch.zeros(4, dtype=torch.int64, device=dev)
+    # mala_fwd: 1 launch; mala_bwd: pre-pass, main kernel, dQ conversion
+    launches_per_step = 4
 
-    def step(tau, st=None):
+    def step(tau, st=None, bst=None, ev_f=None, ev_b=None):
+        if ev_f is not None:
+            ev_f[0].record(stream)
         mala.mala_fwd(q, k, v, tau, TILE, TILE, o=o, lse=lse, keep_mask=keep, stats=st)
+        if ev_f is not None:
+            ev_f[1].record(stream)
+            ev_b[0].record(stream)
+        mala.mala_bwd(q, k, v, o, do, lse, tau, keep, dq=dq, dk=dk, dv=dv, stats=bst)
+        if ev_b is not None:
+            ev_b[1].record(stream)
 
     # one measured step for the executed-work counts
     stats.zero_()
-    step(TAU, stats)
+    bstats.zero_()
+    step(TAU, stats, bstats)
     mala.check_device_error()
     tested, kept, slots = (int(x) for x in stats.cpu().tolist()[:3])
+    b_visit, b_kept, b_slots = (int(x) for x in bstats.cpu().tolist()[:3])
     fwd_flops = tile_flops(d) * (tested + kept)
+    bwd_flops = tile_flops(d) * (b_visit + 4 * b_kept)
 
     for _ in range(args.warmup):
         step(TAU)
     torch.cuda.synchronize()
 
-    # per-launch kernel time with events on the launching stream
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    # per-launch kernel times with events on the launching stream
+    mk = lambda: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    evf = [mk() for _ in range(args.steps)]
+    evb = [mk() for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -165,15 +180,14 @@ def run_mala(args):
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
-        for s in range(args.steps):
-            ev[s][0].record(stream)
-            step(TAU)
-            ev[s][1].record(stream)
+        for s_ in range(args.steps):
+            step(TAU, ev_f=evf[s_], ev_b=evb[s_])
         t1.record(stream)
         torch.cuda.synchronize()
     elapsed = t0.elapsed_time(t1) / 1e3
     mala.check_device_error()
-    fwd_times = [a.elapsed_time(b) / 1e3 for a, b in ev]
+    fwd_times = [a.elapsed_time(b_) / 1e3 for a, b_ in evf]
+    bwd_times = [a.elapsed_time(b_) / 1e3 for a, b_ in evb]
     if world > 1:
         tt = torch.tensor([elapsed], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -191,37 +205,48 @@ def run_mala(args):
 
     # dense comparison: the same kernels at tau = 0
     stats.zero_()
-    step(0.0, stats)
+    bstats.zero_()
+    step(0.0, stats, bstats)
     d_tested, d_kept, _ = (int(x) for x in stats.cpu().tolist()[:3])
+    db_visit, db_kept, _ = (int(x) for x in bstats.cpu().tolist()[:3])
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_dense = max(1, args.steps // 2)
     e0.record(stream)
-    for _ in range(max(1, args.steps // 2)):
+    for _ in range(n_dense):
         step(0.0)
     e1.record(stream)
     torch.cuda.synchronize()
-    dense_s = e0.elapsed_time(e1) / 1e3 / max(1, args.steps // 2)
+    dense_s = e0.elapsed_time(e1) / 1e3 / n_dense
+    dense_flops = tile_flops(d) * (d_tested + d_kept + db_visit + 4 * db_kept)
 
-    # end to end through the public API with pinned host buffers
-    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v"))
-    d2h = o_h.numel() * o_h.element_size()
+    # end to end through the public API with pinned host buffers: inputs in,
+    # forward + backward, output and gradients out, every step
+    outs_h = {n: torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for n, x in
+              (("o", o), ("dq", dq), ("dk", dk), ("dv", dv))}
+    h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v", "do"))
+    d2h = sum(x.numel() * x.element_size() for x in outs_h.values())
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(args.steps):
-        qd = host["q"].to(dev, non_blocking=True)
-        kd = host["k"].to(dev, non_blocking=True)
-        vd = host["v"].to(dev, non_blocking=True)
-        od, _, _ = mala.mala_fwd(qd, kd, vd, TAU, TILE, TILE, with_mask=False)
-        o_h.copy_(od, non_blocking=True)
+        qd, kd, vd, dod = (host[n].to(dev, non_blocking=True) for n in ("q", "k", "v", "do"))
+        od, lsed, kmd = mala.mala_fwd(qd, kd, vd, TAU, TILE, TILE)
+        dqd, dkd, dvd, _ = mala.mala_bwd(qd, kd, vd, od, dod, lsed, TAU, kmd)
+        for n_, x in (("o", od), ("dq", dqd), ("dk", dkd), ("dv", dvd)):
+            outs_h[n_].copy_(x, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_s = e0.elapsed_time(e1) / 1e3
 
     peaks = _peaks()
-    kern_s = statistics.mean(fwd_times)
-    achieved = fwd_flops / kern_s / 1e12
+    dec = None if args.no_decode else bench_decode(args, dev, stream, peaks)
+    kern_f = statistics.mean(fwd_times)
+    kern_b = statistics.mean(bwd_times)
+    ach_f = fwd_flops / kern_f / 1e12
+    ach_b = bwd_flops / kern_b / 1e12
     peak = peaks["bf16_tflops_sustained"]
+    dom = ("mala_bwd (pre + mala_bwd_tc_kernel + dQ conversion)", ach_b) if kern_b >= kern_f \
+        else ("mala_fwd_tc_kernel<128>", ach_f)
     res = {
         "metric": METRIC,
         "value": value,
@@ -234,17 +259,21 @@ def run_mala(args):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic, seeded (gqa_32k recipe: diffuse / local / retrieval head thirds)",
+        "data": "synthetic, seeded (gqa_32k recipe: diffuse / local / retrieval head thirds; dO ~ N(0,1))",
         "config": {"workload": WORKLOAD, "batch": B, "heads_q": Hq, "heads_kv": Hkv, "seqlen": N,
-                   "head_dim": d, "block_q": TILE, "block_k": TILE, "tau": TAU, "pass": "fwd",
-                   "l2": "inputs (0.4 GB) larger than L2; no flush"},
-        "fwd": {"ms": kern_s * 1e3, "tflops_executed": achieved, "tiles_tested": tested,
-                "tiles_kept": kept, "kept_fraction": kept / tested,
+                   "head_dim": d, "block_q": TILE, "block_k": TILE, "tau": TAU, "pass": "fwd+bwd",
+                   "l2": "inputs (0.7 GB) larger than L2; no flush"},
+        "tflops_executed": (fwd_flops + bwd_flops) / (elapsed / args.steps / world) / 1e12,
+        "fwd": {"ms": kern_f * 1e3, "tflops_executed": ach_f, "frac_of_peak": ach_f / peak,
+                "tiles_tested": tested, "tiles_kept": kept, "kept_fraction": kept / tested,
                 "slots_per_query": slots / (B * Hq * N)},
+        "bwd": {"ms": kern_b * 1e3, "tflops_executed": ach_b, "frac_of_peak": ach_b / peak,
+                "tiles_visited": b_visit, "tiles_kept": b_kept, "kept_fraction": b_kept / max(b_visit, 1),
+                "slots_per_query": b_slots / (B * Hq * N)},
         "tau0": {"ms_per_step": dense_s * 1e3, "tokens_per_s": B * N * world / dense_s,
-                 "tflops_executed": tile_flops(d) * (d_tested + d_kept) / dense_s / 1e12},
-        "roofline": {"bound": "tensor", "kernel": "mala_fwd_tc_kernel<128>", "achieved": achieved,
-                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                 "tflops_executed": dense_flops / dense_s / 1e12},
+        "roofline": {"bound": "tensor", "kernel": dom[0], "achieved": dom[1],
+                     "peak": peak, "unit": "TFLOP/s", "frac": dom[1] / peak,
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained",
                      "traffic": None},
         "e2e": {"value": B * N * args.steps / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -252,6 +281,8 @@ def run_mala(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
+    if dec is not None:
+        res["decode"] = dec
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
     if world > 1:
@@ -261,30 +292,101 @@ def run_mala(args):
         print(json.dumps(res), flush=True)
 
 
+def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072):
+    """Split-KV decode on the largest decode workload (batch 64, 32 query
+    heads, 8 KV heads, d = 128, bf16 cache of seqlen_k keys, tau = 0.05).
+    The 34 GB cache is drawn on the device with the decode recipe (sink key,
+    16 needles per sequence). HBM roofline on the bytes actually read:
+    every K tile plus the V tiles some head retained, plus the queries and
+    the split partials written and read back."""
+    import torch
+    from tile_skipping_causal_b200 import mala, synth
+
+    w = synth.decode_workload(args.decode_seqlen or seqlen_k)
+    q = synth.make_decode_query(w, SEED).to(dev)
+    k, v = synth.fill_decode_cache(w, SEED, q.cpu(), dev, slices=[])
+    stats = torch.zeros(4, dtype=torch.int64, device=dev)
+    o, lse, keep, P = mala.mala_decode(q, k, v, w.tau, 128, 0, stats=stats)
+    mala.check_device_error()
+    tested, vread, kept_heads = (int(x) for x in stats.cpu().tolist()[:3])
+    out = torch.empty_like(q)
+    l2 = torch.empty((w.batch, w.heads_q), dtype=torch.float32, device=dev)
+    km = torch.empty_like(keep)
+    workspace = torch.empty(w.batch * w.heads_q * P * 129 * 4 + 256, dtype=torch.uint8, device=dev)
+
+    def call():
+        mala.mala_decode(q, k, v, w.tau, 128, P, o=out, lse=l2, keep_mask=km, workspace=workspace)
+
+    for _ in range(max(3, args.warmup)):
+        call()
+    torch.cuda.synchronize()
+    n = max(5, args.steps // 2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    mala.check_device_error()
+    t = e0.elapsed_time(e1) / 1e3 / n
+    d = w.head_dim
+    kbytes = w.batch * w.heads_kv * w.seqlen_k * d * 2
+    vbytes = vread * 128 * d * 2
+    other = w.batch * w.heads_q * d * 2 * 2 + (w.batch * w.heads_q * P * (d + 1) * 4 * 2 if P > 1 else 0)
+    total = kbytes + vbytes + other
+    gbs = total / t / 1e9
+    del k, v
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "batch": w.batch, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
+            "seqlen_k": w.seqlen_k, "tau": w.tau, "splits": P, "ms": t * 1e3,
+            "tokens_per_s": w.batch / t, "tiles_tested": tested, "v_tiles_read": vread,
+            "v_read_fraction": vread / tested, "head_tiles_kept_fraction": kept_heads / (tested * w.group),
+            "bytes_read_per_call": kbytes + vbytes + w.batch * w.heads_q * d * 2,
+            "roofline": {"bound": "hbm", "kernel": "mala_decode_split_kernel", "achieved": gbs,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "peak_source": f"{peaks['source']} hbm_gbs", "traffic": None}}
+
+
+_ORACLE_INPUTS = {}
+
+
 def _oracle_sample(budget_s: float):
     """Time the fp64 oracle on a seeded random sample of query blocks of the
-    bench workload; returns (rows processed, seconds, blocks)."""
+    bench workload: for each sampled (head, query block) the forward over all
+    its causal key tiles and the backward work of the same tiles (its dQ rows
+    and its share of dK/dV). Returns (rows processed, seconds, blocks)."""
     import numpy as np
     from oracle import mala_oracle as orc
     from tile_skipping_causal_b200 import synth
 
     w = synth.WORKLOADS[WORKLOAD]
-    t = synth.make_prefill(w, SEED)
-    q, k, v = t["q"], t["k"], t["v"]
+    if "t" not in _ORACLE_INPUTS:
+        _ORACLE_INPUTS["t"] = synth.make_prefill(w, SEED, with_do=True)
+    t = _ORACLE_INPUTS["t"]
+    q, k, v, do = t["q"], t["k"], t["v"], t["do"]
     N, G = w.seqlen, w.group
+    nb_ = N // TILE
     rng = np.random.default_rng(0)
     rows = 0
     t0 = time.perf_counter()
     nb = 0
     while time.perf_counter() - t0 < budget_s:
         h = int(rng.integers(0, w.heads_q))
-        i = int(rng.integers(0, N // TILE))
-        Q = q[0, i * TILE:(i + 1) * TILE, h].double().numpy()
+        i = int(rng.integers(0, nb_))
+        q0, q1 = i * TILE, (i + 1) * TILE
+        Qh = q[0, :, h].double().numpy()
         K = k[0, :, h // G].double().numpy()
         V = v[0, :, h // G].double().numpy()
-        st = orc.forward_block(Q, np.arange(i * TILE, (i + 1) * TILE), K, V, TILE, TAU,
-                               orc.causal_tiles((i + 1) * TILE - 1, TILE, N // TILE))
-        orc.finalize(st)
+        st = orc.forward_block(Qh[q0:q1], np.arange(q0, q1), K, V, TILE, TAU,
+                               orc.causal_tiles(q1 - 1, TILE, nb_))
+        Ob, zb = orc.finalize(st)
+        O = np.zeros_like(Qh)
+        z = np.zeros(N)
+        O[q0:q1], z[q0:q1] = Ob, zb
+        fm = np.zeros((nb_, nb_), dtype=bool)
+        fm[i, :i + 1] = [st["keep"][j] for j in range(i + 1)]
+        orc.backward_head(Qh, K, V, O, do[0, :, h].double().numpy(), z, TILE, TILE, TAU, fm,
+                          qblocks=[i])
         rows += TILE
         nb += 1
     return rows, time.perf_counter() - t0, nb
@@ -301,8 +403,9 @@ def _threads():
 def cpu_baseline(seconds: float = 15.0):
     rows, secs, nb = _oracle_sample(seconds)
     return {"value": rows / secs, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
-            "sample": f"{nb} random query blocks (128 rows, all their causal key tiles) of the "
-                      f"{WORKLOAD} workload at tau={TAU}, forward, fp64 numpy, {secs:.1f} s"}
+            "sample": f"{nb} random query blocks (128 rows, forward over all their causal key tiles "
+                      f"and the backward of the same tiles) of the {WORKLOAD} workload at tau={TAU}, "
+                      f"fp64 numpy, {secs:.1f} s"}
 
 
 def run_reference(args):
@@ -325,7 +428,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic, seeded (gqa_32k recipe)",
         "config": {"workload": WORKLOAD, "batch": 1, "heads_q": 32, "heads_kv": 8, "seqlen": 32768,
-                   "head_dim": 128, "block_q": TILE, "block_k": TILE, "tau": TAU, "pass": "fwd"},
+                   "head_dim": 128, "block_q": TILE, "block_k": TILE, "tau": TAU, "pass": "fwd+bwd"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
                          "sample": f"{args.steps} steps of random 128-row query blocks, "
                                    f"{secs_total:.1f} s total"},
@@ -344,12 +447,24 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="shrink N (same recipe); for profiling captures only")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement")
+    ap.add_argument("--decode-seqlen", type=int, default=None,
+                    help="decode cache length (default 131072); for profiling captures")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode measurement (profiling captures)")
     ap.add_argument("--no-extras", action="store_true",
                     help="time the step only (no tau=0, e2e, baseline); for profiling captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         run_reference(args)
+    elif args.decode_only:
+        import torch
+        from tile_skipping_causal_b200 import mala
+        mala.load_library()
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps(bench_decode(args, dev, torch.cuda.current_stream(), _peaks())), flush=True)
     else:
         run_mala(args)
 

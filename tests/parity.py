@@ -166,3 +166,141 @@ def check_decode(q, k, v, o, lse, keep_words, tau, P, B_k=128, heads=None, rep=N
             check_decode_head(f64(q[b, 0, h]), K, V, B_k, tau, P, keep[b, h], o_c[b, 0, h],
                               float(lse_c[b, h]), rep, f"decode b={b} h={h}")
     return rep
+
+
+def oracle_forward_replaying(q64, k64, v64, b, h, G, blocks, gpu_keep_bh, B_q, B_k, tau, rep=None):
+    """Oracle O and z for query blocks ``blocks`` of head (b, h), with the
+    GPU's forward decisions forced; every forced decision that differs from
+    the oracle's own must lie inside the margin band. Returns full-length
+    O [N, d] and z [N] arrays (NaN outside the blocks)."""
+    Q, K, V = q64[b, :, h], k64[b, :, h // G], v64[b, :, h // G]
+    N = Q.shape[0]
+    nKB = orc.num_blocks(N, B_k)
+    O = np.full((N, V.shape[1]), np.nan)
+    z = np.full(N, np.nan)
+    for i in blocks:
+        q0, q1 = i * B_q, min((i + 1) * B_q, N)
+        tiles = orc.causal_tiles(q1 - 1, B_k, nKB)
+        gdec = {j: bool(gpu_keep_bh[i, j]) for j in tiles}
+        st = orc.forward_block(Q[q0:q1], np.arange(q0, q1), K, V, B_k, tau, tiles, replay=gdec)
+        for j in tiles:
+            mj = st["margin"][j]
+            if gdec[j] != (mj <= 0.0):
+                assert abs(mj) <= MARGIN_BAND, f"fwd b={b} h={h} i={i} tile {j}: margin {mj:.3e}"
+                if rep is not None:
+                    rep["fwd_band_flips"] = rep.get("fwd_band_flips", 0) + 1
+        O[q0:q1], z[q0:q1] = orc.finalize(st)
+    return O, z
+
+
+def as_operator_outputs(O, z):
+    """The forward operator emits O in bf16 and the log-normaliser in fp32;
+    the backward consumes exactly those. Round the oracle's fp64 values the
+    same way before they feed the oracle's backward (D = rowsum(dO o O) is a
+    cancelling difference for sharp rows, so the O precision matters)."""
+    Ob = torch.from_numpy(np.ascontiguousarray(O)).to(torch.bfloat16).to(torch.float64).numpy()
+    zf = np.asarray(z, dtype=np.float32).astype(np.float64)
+    return Ob, zf
+
+
+def check_bwd_blocks(q, k, v, do, fwd_keep_words, bwd_keep_words, dq, dk, dv, tau,
+                     kv_samples=None, q_samples=None, B_q=128, B_k=128):
+    """Backward parity. kv_samples: (b, hk, j) key blocks whose dK/dV rows are
+    checked (None = all); q_samples: (b, h, i) query blocks whose dQ rows are
+    checked (None = all). Gradients by relative Frobenius error per block;
+    backward decisions by the margin band."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    nQB, nKB = orc.num_blocks(N, B_q), orc.num_blocks(N, B_k)
+    fkeep = mala.unpack_mask(fwd_keep_words, nKB)
+    bkeep = mala.unpack_mask(bwd_keep_words, nKB) if bwd_keep_words is not None else None
+    q64, k64, v64, do64 = f64(q), f64(k), f64(v), f64(do)
+    dq64, dk64, dv64 = f64(dq), f64(dk), f64(dv)
+    if kv_samples is None:
+        kv_samples = [(b, hk, j) for b in range(B) for hk in range(Hkv) for j in range(nKB)]
+    if q_samples is None:
+        q_samples = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(nQB)]
+    worst = 0.0
+    rep = {}
+    cache = {}
+    err2 = {"dQ": 0.0, "dK": 0.0, "dV": 0.0}
+    ref2 = {"dQ": 0.0, "dK": 0.0, "dV": 0.0}
+
+    def fwd_rows(b, h, blocks):
+        key = (b, h)
+        O, z = cache.get(key, (None, None))
+        need = [i for i in blocks if O is None or np.isnan(z[i * B_q])]
+        if need:
+            O2, z2 = oracle_forward_replaying(q64, k64, v64, b, h, G, need, fkeep[b, h], B_q, B_k, tau, rep)
+            if O is None:
+                O, z = O2, z2
+            else:
+                sel = ~np.isnan(z2)
+                O[sel], z[sel] = O2[sel], z2[sel]
+            cache[key] = (O, z)
+        return as_operator_outputs(*cache[key])
+
+    def check_bmask(b, h, bk_ref, bm_ref, blocks_i, blocks_j):
+        if bkeep is None:
+            return
+        for i in blocks_i:
+            for j in blocks_j:
+                if np.isnan(bm_ref[i, j]):
+                    continue
+                if bool(bkeep[b, h, i, j]) != bool(bk_ref[i, j]):
+                    assert abs(bm_ref[i, j]) <= MARGIN_BAND, \
+                        f"bwd b={b} h={h} tile ({i},{j}): margin {bm_ref[i, j]:.3e}"
+
+    for (b, hk, j) in kv_samples:
+        k0, k1 = j * B_k, min((j + 1) * B_k, N)
+        dK = np.zeros((k1 - k0, d))
+        dV = np.zeros((k1 - k0, d))
+        for h in range(hk * G, (hk + 1) * G):
+            blocks = [i for i in range(j, nQB) if fkeep[b, h, i, j]]
+            if not blocks:
+                continue
+            O, z = fwd_rows(b, h, blocks)
+            dQh, dKh, dVh, bk_ref, bm_ref = orc.backward_head(
+                q64[b, :, h], k64[b, :, hk], v64[b, :, hk], O, do64[b, :, h], z, B_q, B_k, tau,
+                fkeep[b, h], kblocks=[j], qblocks=blocks)
+            dK += dKh[k0:k1]
+            dV += dVh[k0:k1]
+            check_bmask(b, h, bk_ref, bm_ref, blocks, [j])
+        for name, got, ref in (("dK", dk64[b, k0:k1, hk], dK), ("dV", dv64[b, k0:k1, hk], dV)):
+            assert np.isfinite(got).all(), f"{name} b={b} hk={hk} j={j}: non-finite"
+            if np.linalg.norm(ref) == 0.0:
+                # an exactly cancelling reference (e.g. a single key: dS = dP - D = 0)
+                # leaves only fp32 summation-order residue on the GPU
+                assert np.abs(got).max() <= 1e-3, f"{name} b={b} hk={hk} j={j}: expected ~zeros"
+                continue
+            err2[name] += float(np.sum((got - ref) ** 2))
+            ref2[name] += float(np.sum(ref ** 2))
+            worst = max(worst, rel_fro(got, ref))
+
+    for (b, h, i) in q_samples:
+        q0, q1 = i * B_q, min((i + 1) * B_q, N)
+        O, z = fwd_rows(b, h, [i])
+        dQh, _, _, bk_ref, bm_ref = orc.backward_head(
+            q64[b, :, h], k64[b, :, h // G], v64[b, :, h // G], O, do64[b, :, h], z, B_q, B_k, tau,
+            fkeep[b, h], qblocks=[i])
+        check_bmask(b, h, bk_ref, bm_ref, [i], range(0, i + 1))
+        got, ref = dq64[b, q0:q1, h], dQh[q0:q1]
+        assert np.isfinite(got).all(), f"dQ b={b} h={h} i={i}: non-finite"
+        if np.linalg.norm(ref) == 0.0:
+            assert np.abs(got).max() <= 1e-3, f"dQ b={b} h={h} i={i}: expected ~zeros"
+            continue
+        err2["dQ"] += float(np.sum((got - ref) ** 2))
+        ref2["dQ"] += float(np.sum(ref ** 2))
+        worst = max(worst, rel_fro(got, ref))
+    # the tolerance is a relative Frobenius error of each gradient tensor
+    # (over the checked rows); single blocks whose gradient nearly cancels
+    # can carry a larger relative error without mattering for the tensor
+    for name in err2:
+        if ref2[name] > 0.0:
+            e = (err2[name] / ref2[name]) ** 0.5
+            rep[name] = e
+            assert e <= GRAD_RFE, f"{name}: rel. Frobenius error {e:.3e} over the checked rows"
+    rep["worst_block_rel_fro"] = worst
+    rep["worst_rel_fro"] = max([rep[n] for n in err2 if n in rep] or [0.0])
+    return rep

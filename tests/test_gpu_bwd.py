@@ -1,0 +1,153 @@
+"""GPU parity of mala_bwd (Algorithm 2 with forward-mask replay) against the
+fp64 oracle, through the C ABI."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import mala_oracle as orc
+from tile_skipping_causal_b200 import mala, synth
+from tests.parity import check_bwd_blocks
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+SEED = 42
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from tile_skipping_causal_b200 import build
+    build.build()
+    mala.load_library()
+
+
+def _fwd_bwd(t, tau, pure=False, **kw):
+    o, lse, keep = mala.mala_fwd(t["q"], t["k"], t["v"], tau, 128, 128)
+    dq, dk, dv, bkeep = mala.mala_bwd(t["q"], t["k"], t["v"], o, t["do"], lse, tau,
+                                      None if pure else keep, with_bwd_mask=True, **kw)
+    mala.check_device_error()
+    return o, lse, keep, dq, dk, dv, bkeep
+
+
+def _run(w, seed=SEED, **kw):
+    t = synth.make_prefill(w, seed, with_do=True, **kw)
+    return {n: x.to(DEV) for n, x in t.items()}
+
+
+@pytest.mark.parametrize("tau", [0.1, 1.0])
+def test_train_recipe_reduced_all_blocks(tau):
+    t = _run(synth.WORKLOADS["train_8k"], batch=1, seqlen=1000)
+    o, lse, keep, dq, dk, dv, bkeep = _fwd_bwd(t, tau)
+    rep = check_bwd_blocks(t["q"], t["k"], t["v"], t["do"], keep, bkeep, dq, dk, dv, tau)
+    assert rep["worst_rel_fro"] < 3e-2
+
+
+@pytest.mark.parametrize("name,tau", [("train_8k", 0.1), ("train_8k", 1.0), ("gqa_32k", 0.2)])
+def test_backward_on_oracle_forward_outputs(name, tau):
+    """mala_bwd alone: O (bf16), LSE (fp32) and the forward mask all come
+    from the oracle's forward, so both sides consume identical inputs."""
+    import numpy as np
+    from tests.parity import as_operator_outputs, f64, rel_fro
+    w = synth.WORKLOADS[name]
+    t = synth.make_prefill(w, SEED, with_do=True, batch=1, seqlen=640)
+    q64, k64, v64, do64 = (f64(t[n]) for n in ("q", "k", "v", "do"))
+    O, lse, keep, _ = orc.forward(q64, k64, v64, 128, 128, tau)
+    Ob, zf = as_operator_outputs(O, lse)
+    ref = orc.backward(q64, k64, v64, Ob, do64, zf, 128, 128, tau, keep)
+    dev = {n: x.to(DEV) for n, x in t.items()}
+    o_in = torch.from_numpy(Ob).to(torch.bfloat16).to(DEV)
+    lse_in = torch.from_numpy(zf).float().to(DEV)
+    keep_in = torch.from_numpy(mala.pack_mask(keep)).to(DEV)
+    dq, dk, dv, bkeep = mala.mala_bwd(dev["q"], dev["k"], dev["v"], o_in, dev["do"], lse_in, tau, keep_in,
+                                      with_bwd_mask=True)
+    mala.check_device_error()
+    for got, r, name in ((dq, ref[0], "dQ"), (dk, ref[1], "dK"), (dv, ref[2], "dV")):
+        e = rel_fro(f64(got), r)
+        assert e <= 3e-2, f"{name} rel. Frobenius error {e:.3e}"
+    # decisions: equal except inside the margin band
+    nQB = 5
+    gb = mala.unpack_mask(bkeep, nQB)
+    Hq, G = w.heads_q, w.group
+    for h in range(Hq):
+        _, _, _, kh, mh = orc.backward_head(q64[0, :, h], k64[0, :, h // G], v64[0, :, h // G], Ob[0, :, h],
+                                            do64[0, :, h], zf[0, h], 128, 128, tau, keep[0, h])
+        diff = gb[0, h] != kh
+        assert not diff.any() or np.abs(mh[diff]).max() <= 1e-3
+
+
+def test_gqa_recipe_reduced_all_blocks():
+    t = _run(synth.WORKLOADS["gqa_32k"], seqlen=768)
+    o, lse, keep, dq, dk, dv, bkeep = _fwd_bwd(t, 0.2)
+    check_bwd_blocks(t["q"], t["k"], t["v"], t["do"], keep, bkeep, dq, dk, dv, 0.2)
+
+
+def test_tau_zero_is_dense_gradient():
+    t = _run(synth.WORKLOADS["train_8k"], batch=1, seqlen=640)
+    o, lse, keep, dq, dk, dv, bkeep = _fwd_bwd(t, 0.0)
+    nQB = 5
+    m = mala.unpack_mask(bkeep, nQB)
+    assert (m == np.tril(np.ones((nQB, nQB), dtype=bool))[None, None]).all()
+    check_bwd_blocks(t["q"], t["k"], t["v"], t["do"], keep, bkeep, dq, dk, dv, 0.0)
+
+
+def test_tau_inf_gradients_vanish():
+    t = _run(synth.WORKLOADS["train_8k"], batch=1, seqlen=512)
+    o, lse, keep, dq, dk, dv, bkeep = _fwd_bwd(t, math.inf)
+    assert not mala.unpack_mask(bkeep, 4).any()
+    for g in (dq, dk, dv):
+        assert g.abs().max().item() == 0.0
+
+
+def test_pure_backward_equals_mask_replay_and_nests():
+    """Without the stored mask every legal tile is re-tested: the retained
+    set nests inside the forward's (up to the margin band) and the gradients
+    match the mask-replay run."""
+    t = _run(synth.WORKLOADS["train_8k"], batch=1, seqlen=768)
+    o, lse, keep, dq, dk, dv, bkeep = _fwd_bwd(t, 0.1)
+    _, _, _, dq2, dk2, dv2, bkeep2 = _fwd_bwd(t, 0.1, pure=True)
+    fm = mala.unpack_mask(keep, 6)
+    b1 = mala.unpack_mask(bkeep, 6)
+    b2 = mala.unpack_mask(bkeep2, 6)
+    assert not (b2 & ~fm).any() or (b2 & ~fm).sum() <= 2
+    assert (b1 == (b2 & fm)).all()
+    for a, c in ((dq, dq2), (dk, dk2), (dv, dv2)):
+        assert torch.equal(a, c) or (a.float() - c.float()).norm() <= 1e-2 * c.float().norm()
+
+
+@pytest.mark.parametrize("N", [1, 100, 128, 129, 300])
+def test_edge_lengths_gqa(N):
+    g = torch.Generator().manual_seed(N)
+    B, Hq, Hkv, d = 2, 4, 2, 128
+    t = {"q": (torch.randn(B, N, Hq, d, generator=g) * 3 / math.sqrt(d)).bfloat16().to(DEV),
+         "k": torch.randn(B, N, Hkv, d, generator=g).bfloat16().to(DEV),
+         "v": torch.randn(B, N, Hkv, d, generator=g).bfloat16().to(DEV),
+         "do": torch.randn(B, N, Hq, d, generator=g).bfloat16().to(DEV)}
+    o, lse, keep, dq, dk, dv, bkeep = _fwd_bwd(t, 0.3)
+    check_bwd_blocks(t["q"], t["k"], t["v"], t["do"], keep, bkeep, dq, dk, dv, 0.3)
+
+
+def test_rademacher_probe_direction():
+    """The paper's operator-fidelity protocol drives the backward with a
+    deterministic Rademacher dO."""
+    t = _run(synth.WORKLOADS["train_8k"], batch=1, seqlen=512)
+    t["do"] = synth.rademacher_like(tuple(t["q"].shape), 7).to(DEV)
+    o, lse, keep, dq, dk, dv, bkeep = _fwd_bwd(t, 0.1)
+    check_bwd_blocks(t["q"], t["k"], t["v"], t["do"], keep, bkeep, dq, dk, dv, 0.1)
+
+
+def test_train_8k_full_size_sampled():
+    w = synth.WORKLOADS["train_8k"]
+    t = _run(w)
+    stats = torch.zeros(4, dtype=torch.int64, device=DEV)
+    o, lse, keep, dq, dk, dv, bkeep = _fwd_bwd(t, 0.1, stats=stats)
+    nQB = 64
+    kv = [(0, 0, 63), (1, 9, 60), (3, 15, 50), (2, 4, 62)]
+    qs = [(0, 0, 0), (1, 9, 5), (3, 15, 20), (2, 12, 63)]
+    check_bwd_blocks(t["q"], t["k"], t["v"], t["do"], keep, bkeep, dq, dk, dv, w.taus[0],
+                     kv_samples=kv, q_samples=qs)
+    s = stats.cpu().tolist()
+    fm = mala.unpack_mask(keep, nQB)
+    bm = mala.unpack_mask(bkeep, nQB)
+    assert s[0] == fm.sum() and s[1] == bm.sum()

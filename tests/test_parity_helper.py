@@ -84,3 +84,22 @@ def test_decode_checker_rejects_wrong_decision_and_output():
     o2[0, 0, 3, 5] += 0.3
     with pytest.raises(AssertionError, match="O"):
         parity.check_decode(q, k, v, o2, lse, torch.from_numpy(mala.pack_mask(keep)), 2.0, 1)
+
+
+def test_backward_checker_accepts_oracle_and_rejects_planted_error():
+    t = synth.make_prefill(synth.WORKLOADS["train_8k"], 4, batch=1, seqlen=300, with_do=True)
+    q, k, v, do = t["q"], t["k"], t["v"], t["do"]
+    tau = 0.1
+    O, lse, keep, _ = orc.forward(parity.f64(q), parity.f64(k), parity.f64(v), 128, 128, tau)
+    Ob, zf = parity.as_operator_outputs(O, lse)
+    dq, dk, dv, bkeep = orc.backward(parity.f64(q), parity.f64(k), parity.f64(v), Ob, parity.f64(do), zf,
+                                     128, 128, tau, keep)
+    fw = torch.from_numpy(mala.pack_mask(keep))
+    bw = torch.from_numpy(mala.pack_mask(bkeep))
+    cast = lambda x: torch.from_numpy(x).to(torch.bfloat16)
+    rep = parity.check_bwd_blocks(q, k, v, do, fw, bw, cast(dq), cast(dk), cast(dv), tau)
+    assert rep["worst_rel_fro"] < 1e-2
+    dk_bad = dk.copy()
+    dk_bad[0, :, 3] *= 1.5            # one head of 16 off by 50%: about 12% of the tensor
+    with pytest.raises(AssertionError, match="dK"):
+        parity.check_bwd_blocks(q, k, v, do, fw, bw, cast(dq), cast(dk_bad), cast(dv), tau)

@@ -75,4 +75,40 @@ struct DecodeParams {
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
 size_t decode_smem_bytes();
 
+// Backward (bf16, d = 128, B_q = B_k = 128, N_q = N_k).
+struct BwdParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;   // 4-D maps, box {64, 1, 128, 1}, 128B swizzle
+  const float* zl2;        // [B, Hq, Npad] z log2e
+  const float* t2;         // [B, Hq, Npad] (z + log tau - log L_q) log2e
+  const float* Dv;         // [B, Hq, Npad] rowsum(dO o O)
+  float* dq_acc;           // [B, Hq, nQB, 4, 128, 32] fp32
+  void* dk;
+  void* dv;
+  const uint32_t* fwd_mask;  // [B, Hq, nQB, mask_words] or NULL (visit every legal tile)
+  uint32_t* bwd_mask;        // same layout, zeroed by the host, or NULL
+  int64_t* stats;
+  int* err;
+  int64_t dk_sb, dk_sn, dk_sh, dv_sb, dv_sn, dv_sh;
+  int B, Hq, Hkv, N, Npad, nQB, nKB, mask_words;
+  uint8_t group_size[kMaxKvHeads];
+  uint8_t group_heads[kMaxKvHeads][kMaxGroup];
+};
+
+struct BwdAuxParams {      // pre-pass and dQ conversion
+  const void* o;
+  const void* dout;
+  const float* lse;
+  float* zl2;
+  float* t2;
+  float* Dv;
+  float* dq_acc;
+  void* dq;
+  int64_t o_sb, o_sn, o_sh, do_sb, do_sn, do_sh, dq_sb, dq_sn, dq_sh;
+  int B, Hq, N, Npad, nQB;
+  float log_tau;
+};
+
+cudaError_t launch_bwd(const BwdParams& p, const BwdAuxParams& aux, cudaStream_t stream);
+size_t bwd_smem_bytes();
+
 }  // namespace mala

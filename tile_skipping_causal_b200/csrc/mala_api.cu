@@ -263,18 +263,123 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
 
 // ------------------------------------------------------------------ backward
 
-size_t mala_bwd_workspace_size(const mala_bwd_args* a) {
-  (void)a;
-  return 0;
+namespace {
+
+int bwd_check(const mala_bwd_args* a) {
+  int rc = check_common(a->batch, a->heads_q, a->heads_kv, a->head_dim, a->tau, a->dtype);
+  if (rc) return rc;
+  if (a->dtype != MALA_BF16) return fail(MALA_ERR_UNSUPPORTED, "backward supports bf16 only");
+  if (a->head_dim != 128) return fail(MALA_ERR_UNSUPPORTED, "backward supports head_dim 128 only");
+  if (a->block_q != 128 || a->block_k != 128) return fail(MALA_ERR_UNSUPPORTED, "backward supports 128 x 128 tiles only");
+  if (a->seqlen_q <= 0 || a->seqlen_k <= 0) return fail(MALA_ERR_INVALID_ARG, "sequence lengths must be positive");
+  if (a->seqlen_q != a->seqlen_k) return fail(MALA_ERR_UNSUPPORTED, "causal backward needs seqlen_q == seqlen_k");
+  if (a->seqlen_q > (1 << 30)) return fail(MALA_ERR_UNSUPPORTED, "sequence too long");
+  if (a->heads_kv > mala::kMaxKvHeads) return fail(MALA_ERR_UNSUPPORTED, "heads_kv > %d", mala::kMaxKvHeads);
+  if (!a->lse) return fail(MALA_ERR_INVALID_ARG, "lse is NULL");
+  if ((rc = check_tensor("q", a->q, a->q_stride, 2, 128, a->heads_q))) return rc;
+  if ((rc = check_tensor("k", a->k, a->k_stride, 2, 128, a->heads_kv))) return rc;
+  if ((rc = check_tensor("v", a->v, a->v_stride, 2, 128, a->heads_kv))) return rc;
+  if ((rc = check_tensor("o", a->o, a->o_stride, 2, 128, a->heads_q))) return rc;
+  if ((rc = check_tensor("dout", a->dout, a->do_stride, 2, 128, a->heads_q))) return rc;
+  if ((rc = check_tensor("dq", a->dq, a->dq_stride, 2, 128, a->heads_q))) return rc;
+  if ((rc = check_tensor("dk", a->dk, a->dk_stride, 2, 128, a->heads_kv))) return rc;
+  if ((rc = check_tensor("dv", a->dv, a->dv_stride, 2, 128, a->heads_kv))) return rc;
+  return MALA_OK;
 }
 
-int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* stream) {
-  (void)workspace;
-  (void)ws_bytes;
-  (void)stream;
+// workspace: zl2, t2, D ([B, Hq, Npad] fp32 each) then the blocked dQ accumulator
+size_t bwd_ws_bytes(const mala_bwd_args* a) {
+  const size_t npad = static_cast<size_t>((a->seqlen_q + 127) / 128) * 128;
+  const size_t rows = static_cast<size_t>(a->batch) * a->heads_q * npad;
+  return rows * 3 * sizeof(float) + rows * 128 * sizeof(float) + 256;
+}
+
+}  // namespace
+
+size_t mala_bwd_workspace_size(const mala_bwd_args* a) {
+  if (!a || bwd_check(a) != MALA_OK) return 0;
+  return bwd_ws_bytes(a);
+}
+
+int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* stream_) {
   g_msg[0] = 0;
   if (!a) return fail(MALA_ERR_INVALID_ARG, "args is NULL");
-  return fail(MALA_ERR_UNSUPPORTED, "backward kernel not built yet");
+  int rc = bwd_check(a);
+  if (rc) return rc;
+  const size_t need = bwd_ws_bytes(a);
+  if (!workspace || ws_bytes < need) return fail(MALA_ERR_WORKSPACE, "backward workspace of %zu bytes needed", need);
+  if (!aligned16(workspace)) return fail(MALA_ERR_INVALID_ARG, "workspace misaligned");
+  const int N = static_cast<int>(a->seqlen_q);
+  const int nQB = (N + 127) / 128;
+  const int Npad = nQB * 128;
+  const size_t rows = static_cast<size_t>(a->batch) * a->heads_q * Npad;
+
+  mala::BwdParams p;
+  memset(&p, 0, sizeof(p));
+  uint8_t kv_of_q[mala::kMaxHeads];
+  if ((rc = head_map(a->q_to_kv, a->heads_q, a->heads_kv, kv_of_q))) return rc;
+  for (int64_t h = 0; h < a->heads_q; ++h) {
+    const int hk = kv_of_q[h];
+    if (p.group_size[hk] >= mala::kMaxGroup)
+      return fail(MALA_ERR_UNSUPPORTED, "more than %d query heads share KV head %d", mala::kMaxGroup, hk);
+    p.group_heads[hk][p.group_size[hk]++] = static_cast<uint8_t>(h);
+  }
+  if ((rc = make_map_bf16(&p.tm_q, a->q, a->batch, N, a->heads_q, 128, a->q_stride, 128))) return rc;
+  if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, N, a->heads_kv, 128, a->k_stride, 128))) return rc;
+  if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, N, a->heads_kv, 128, a->v_stride, 128))) return rc;
+  if ((rc = make_map_bf16(&p.tm_do, a->dout, a->batch, N, a->heads_q, 128, a->do_stride, 128))) return rc;
+  float* ws = static_cast<float*>(workspace);
+  p.zl2 = ws;
+  p.t2 = ws + rows;
+  p.Dv = ws + 2 * rows;
+  p.dq_acc = ws + 3 * rows;
+  p.dk = a->dk;
+  p.dv = a->dv;
+  p.fwd_mask = a->keep_mask;
+  p.bwd_mask = a->bwd_keep_mask;
+  p.stats = a->stats;
+  p.err = device_error_ptr();
+  if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
+  p.dk_sb = a->dk_stride[0]; p.dk_sn = a->dk_stride[1]; p.dk_sh = a->dk_stride[2];
+  p.dv_sb = a->dv_stride[0]; p.dv_sn = a->dv_stride[1]; p.dv_sh = a->dv_stride[2];
+  p.B = static_cast<int>(a->batch);
+  p.Hq = static_cast<int>(a->heads_q);
+  p.Hkv = static_cast<int>(a->heads_kv);
+  p.N = N;
+  p.Npad = Npad;
+  p.nQB = nQB;
+  p.nKB = nQB;
+  p.mask_words = (nQB + 31) / 32;
+
+  mala::BwdAuxParams x;
+  memset(&x, 0, sizeof(x));
+  x.o = a->o;
+  x.dout = a->dout;
+  x.lse = a->lse;
+  x.zl2 = ws;
+  x.t2 = ws + rows;
+  x.Dv = ws + 2 * rows;
+  x.dq_acc = ws + 3 * rows;
+  x.dq = a->dq;
+  x.o_sb = a->o_stride[0]; x.o_sn = a->o_stride[1]; x.o_sh = a->o_stride[2];
+  x.do_sb = a->do_stride[0]; x.do_sn = a->do_stride[1]; x.do_sh = a->do_stride[2];
+  x.dq_sb = a->dq_stride[0]; x.dq_sn = a->dq_stride[1]; x.dq_sh = a->dq_stride[2];
+  x.B = p.B;
+  x.Hq = p.Hq;
+  x.N = N;
+  x.Npad = Npad;
+  x.nQB = nQB;
+  x.log_tau = a->tau == 0.0f ? -INFINITY : logf(a->tau);
+
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (a->bwd_keep_mask) {
+    cudaError_t e = cudaMemsetAsync(a->bwd_keep_mask, 0,
+                                    static_cast<size_t>(a->batch) * a->heads_q * nQB * p.mask_words * 4, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "backward mask clear");
+  }
+  cudaError_t e = mala::launch_bwd(p, x, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+  return MALA_OK;
 }
 
 // ------------------------------------------------------------------ decode
