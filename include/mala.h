@@ -208,6 +208,34 @@ MALA_API size_t mala_decode_workspace_size(const mala_decode_args* args);
 MALA_API int mala_decode(mala_decode_args* args, void* workspace, size_t workspace_bytes,
                 void* stream);
 
+/*
+ * mala_decode_noalloc: mala_decode for callers that cannot allocate device
+ * memory. The paper has no counterpart to this entry point; it exists for
+ * code that is handed only its input and output buffers, such as a plugin
+ * inside a host framework that owns every device allocation and offers no
+ * workspace, or a serving loop that forbids allocation after start-up to
+ * keep its memory footprint fixed. Such callers cannot provide the
+ * workspace that mala_decode needs for its split partials.
+ *
+ * Same arguments, semantics and results as mala_decode, but the split
+ * partials live in a buffer built into the library: a device array of
+ * MALA_DECODE_NOALLOC_SCRATCH_BYTES that every GPU loading the library
+ * holds until the process exits. Nothing is allocated or freed by the call.
+ *   - The partials take batch * heads_q * (128 + 1) * 4 bytes per split.
+ *     num_splits = 0 picks the same split count as mala_decode, lowered
+ *     until the partials fit (down to one split, which needs no scratch); an
+ *     explicit num_splits whose partials do not fit returns
+ *     MALA_ERR_WORKSPACE with the sizes in mala_last_error_message().
+ *   - The first call on each device looks up the buffer's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls share the one buffer, which keeps the last call's contents.
+ *     Calls whose kernels overlap on the GPU (e.g. on different streams
+ *     without ordering) race on it and give wrong results: order them.
+ */
+#define MALA_DECODE_NOALLOC_SCRATCH_BYTES (4u << 20)
+MALA_API int mala_decode_noalloc(mala_decode_args* args, void* stream);
+
 /* Human-readable name of a return code. */
 MALA_API const char* mala_status_string(int status);
 

@@ -498,3 +498,105 @@ int mala_decode(mala_decode_args* a, void* workspace, size_t ws_bytes, void* str
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ decode without allocation
+
+namespace {
+
+// Built-in scratch for mala_decode_noalloc: the split-KV partial outputs and
+// log-normalisers ([B, H_q, P, 128] + [B, H_q, P] fp32). Every GPU that
+// loads the library holds it until the process exits. In host code the name
+// only stands for the symbol; its device address comes from
+// cudaGetSymbolAddress (see decode_noalloc_scratch below).
+static __device__ __align__(256) float g_decode_noalloc_scratch[MALA_DECODE_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+// Device address of the scratch array on the current device, looked up once
+// per device (with that device current) and cached.
+float* decode_noalloc_scratch() {
+  static float* ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+    ptrs[dev] = static_cast<float*>(p);
+  }
+  return ptrs[dev];
+}
+
+}  // namespace
+
+extern "C" int mala_decode_noalloc(mala_decode_args* a, void* stream_) {
+  g_msg[0] = 0;
+  if (!a) return fail(MALA_ERR_INVALID_ARG, "args is NULL");
+  int nKB = 0;
+  int rc = decode_check(a, &nKB);
+  if (rc) return rc;
+  // bytes of partials per split: one 128-float row and one log-normaliser per (batch, head)
+  const size_t per_split = static_cast<size_t>(a->batch) * a->heads_q * (128 + 1) * sizeof(float);
+  const size_t cap = MALA_DECODE_NOALLOC_SCRATCH_BYTES;
+  int P = a->num_splits;
+  if (P > 1 && per_split * P > cap)
+    return fail(MALA_ERR_WORKSPACE,
+                "num_splits=%d needs %zu bytes of scratch; the built-in buffer holds %zu (use fewer splits)",
+                P, per_split * P, cap);
+  if (P == 0) {
+    P = choose_splits(a->batch * a->heads_kv, nKB);
+    while (P > 1 && per_split * P > cap) --P;   // fall back to fewer splits, down to none
+  }
+  float* scratch = nullptr;
+  if (P > 1) {
+    scratch = decode_noalloc_scratch();
+    if (!scratch) return fail(MALA_ERR_CUDA, "cannot resolve the built-in decode scratch buffer");
+  }
+
+  mala::DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  uint8_t kv_of_q[mala::kMaxHeads];
+  if ((rc = head_map(a->q_to_kv, a->heads_q, a->heads_kv, kv_of_q))) return rc;
+  for (int64_t h = 0; h < a->heads_q; ++h) {
+    const int hk = kv_of_q[h];
+    if (p.group_size[hk] >= mala::kMaxGroup)
+      return fail(MALA_ERR_UNSUPPORTED, "more than %d query heads share KV head %d", mala::kMaxGroup, hk);
+    p.group_heads[hk][p.group_size[hk]++] = static_cast<uint8_t>(h);
+  }
+  if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, a->seqlen_k, a->heads_kv, 128, a->k_stride, 128))) return rc;
+  if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, a->seqlen_k, a->heads_kv, 128, a->v_stride, 128))) return rc;
+  p.err = device_error_ptr();
+  if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
+  p.q = a->q;
+  p.o = a->o;
+  p.lse = a->lse;
+  p.keep_mask = a->keep_mask;
+  p.stats = a->stats;
+  if (P > 1) {
+    // the partials need no clearing: every split writes all of its rows
+    // before the merge kernel reads them
+    p.part_o = scratch;
+    p.part_lse = scratch + static_cast<size_t>(a->batch) * a->heads_q * P * 128;
+  }
+  p.q_sb = a->q_stride[0];
+  p.q_sh = a->q_stride[2];
+  p.o_sb = a->o_stride[0];
+  p.o_sh = a->o_stride[2];
+  p.B = static_cast<int>(a->batch);
+  p.Hq = static_cast<int>(a->heads_q);
+  p.Hkv = static_cast<int>(a->heads_kv);
+  p.Nk = static_cast<int>(a->seqlen_k);
+  p.nKB = nKB;
+  p.mask_words = (nKB + 31) / 32;
+  p.num_splits = P;
+  p.log2_tau = a->tau == 0.0f ? -INFINITY : log2f(a->tau);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (a->keep_mask) {
+    cudaError_t e = cudaMemsetAsync(a->keep_mask, 0,
+                                    static_cast<size_t>(a->batch) * a->heads_q * p.mask_words * 4, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "keep mask clear");
+  }
+  cudaError_t e = mala::launch_decode(p, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  a->num_splits = P;
+  return MALA_OK;
+}

@@ -71,7 +71,11 @@ EXPORTS = (
     "mala_fwd", "mala_fwd_workspace_size", "mala_bwd", "mala_bwd_workspace_size",
     "mala_decode", "mala_decode_workspace_size", "mala_status_string",
     "mala_last_error_message", "mala_check_device_error", "mala_version",
+    "mala_decode_noalloc",
 )
+
+# size of the library's built-in decode scratch buffer (include/mala.h)
+DECODE_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 _lib = None
 
@@ -112,6 +116,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mala_check_device_error.restype = ctypes.c_int
     lib.mala_version.argtypes = []
     lib.mala_version.restype = ctypes.c_char_p
+    lib.mala_decode_noalloc.argtypes = [ctypes.POINTER(DecodeArgs), vp]
+    lib.mala_decode_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -294,6 +300,39 @@ def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *,
     if workspace is None or workspace.numel() < ws_n:
         workspace = torch.empty(ws_n, dtype=torch.uint8, device=q.device) if ws_n else None
     _check(lib.mala_decode(ctypes.byref(a), _ptr(workspace), ws_n, _stream(stream)))
+    del keep_alive
+    return o, lse, keep_mask, int(a.num_splits)
+
+
+def mala_decode_noalloc(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *, o=None,
+                        lse=None, keep_mask=None, with_mask: bool = True, stats=None, q_to_kv=None,
+                        stream=None):
+    """mala_decode without a workspace: the library keeps the split partials
+    in its own built-in device buffer (for callers that cannot allocate;
+    calls that overlap on the GPU race on that buffer). Returns the same
+    tuple as :func:`mala_decode`."""
+    lib = load_library()
+    _require_cuda(q, k, v)
+    B, _, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    nKB = -(-Nk // block_k)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
+    if keep_mask is None and with_mask:
+        keep_mask = torch.empty((B, Hq, mask_words(nKB)), dtype=torch.int32, device=q.device)
+    keep_alive, hm = _head_map(q_to_kv)
+    a = DecodeArgs()
+    a.q, a.k, a.v, a.o = _ptr(q), _ptr(k), _ptr(v), _ptr(o)
+    a.lse, a.keep_mask = _ptr(lse), _ptr(keep_mask)
+    a.batch, a.heads_q, a.heads_kv, a.seqlen_k, a.head_dim = B, Hq, Hkv, Nk, d
+    a.q_stride, a.k_stride, a.v_stride, a.o_stride = _strides(q), _strides(k), _strides(v), _strides(o)
+    a.q_to_kv = hm
+    a.block_k = block_k
+    a.tau = float(tau)
+    a.dtype = _dtype_code(q)
+    a.num_splits = int(num_splits)
+    a.stats = _ptr(stats)
+    _check(lib.mala_decode_noalloc(ctypes.byref(a), _stream(stream)))
     del keep_alive
     return o, lse, keep_mask, int(a.num_splits)
 
