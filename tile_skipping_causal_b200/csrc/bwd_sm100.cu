@@ -12,13 +12,19 @@
 // with dQ accumulated in fp32 by bulk reduce-add into a blocked workspace.
 //
 // Roles (192 threads): warps 0-3 compute (thread t owns key row t for
-// S^T, P^T, dP^T, dS^T, dK, dV and query row t for the dQ part), warp 4
-// TMA producer, warp 5 tcgen05 issuer.
-// TMEM: X = cols [0,128) holds S^T, later the tile's dQ part; Y = [128,256)
-// holds dP^T; dK = [256,384); dV = [384,512).
-// Shared memory: K_j, V_j, Q_i, dO_i, P^T and dS^T tiles (bf16, 128-byte
-// swizzle); the P^T tile doubles as the fp32 staging buffer of the dQ
-// reduction once dV has consumed it.
+// S^T, P^T, dP^T, dS^T and query row t for the dQ part), warp 4 TMA
+// producer (polling: Q of the next tiles and dO of retained tiles), warp 5
+// tcgen05 issuer.
+// TMEM: X = cols [0,128): S^T(n), then P^T(n) as packed bf16 in [0,64),
+// read by the dV MMA straight from TMEM; Y = [128,256): dP^T(n), then the
+// tile's dQ part; dK = [256,384); dV = [384,512).
+// Shared memory: K_j, V_j, two Q_i stages (with their row statistics), dO_i,
+// and the dS^T tile, which doubles as the fp32 staging buffer of the dQ
+// reduction once dK and dQ have consumed it.
+//
+// Issue order of the tensor pipe for a retained tile n:
+//   dV(n), dP^T(n) -> Y, S^T(n+1) -> X, dK(n), dQ(n) -> Y
+// while the compute warps run the test and P^T of tile n+1 and drain dQ(n).
 #include <math.h>
 
 #include "kernels.h"
@@ -34,21 +40,21 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTile = kB * kD * 2;       // 32 KB bf16 tile
 constexpr uint32_t kChunk = 16384;            // one 64-column swizzle chunk of 128 rows
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kEndMarker = 0xFFFFFFFFu;
 
 enum Bar {
-  kKVFull, kQFull, kQEmpty, kSFull, kXFree, kDecFull, kDecEmpty, kDoFull, kDoEmpty,
-  kPtFull, kPtFree, kDpFull, kDsFull, kDsFree, kDqFull, kDone, kNumBars
+  kKVFull, kQFull, kQEmpty = kQFull + 2, kSFull = kQEmpty + 2, kXRead, kDecFull, kDecEmpty,
+  kDoFull, kDoEmpty, kPtFull, kDvDone, kYFree, kDpFull, kDsFull, kDqFull, kDone, kNumBars
 };
 
 struct Smem {
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + kTile;
-  static constexpr uint32_t kQ = kV + kTile;
-  static constexpr uint32_t kDO = kQ + kTile;
-  static constexpr uint32_t kPT = kDO + kTile;
-  static constexpr uint32_t kDS = kPT + kTile;
-  static constexpr uint32_t kStats = kDS + kTile;          // zl2[128], t2[128], D[128]
-  static constexpr uint32_t kBars = kStats + 3 * 128 * 4;
+  static constexpr uint32_t kQ = kV + kTile;                // 2 stages
+  static constexpr uint32_t kDO = kQ + 2 * kTile;
+  static constexpr uint32_t kDS = kDO + kTile;
+  static constexpr uint32_t kStats = kDS + kTile;           // [2 stages][zl2, t2, D][128]
+  static constexpr uint32_t kBars = kStats + 2 * 3 * 128 * 4;
   static constexpr uint32_t kMisc = kBars + kNumBars * 8;
   static constexpr uint32_t kEnd = kMisc + 64;
   static constexpr uint32_t kAlloc = kEnd + 1024;
@@ -61,16 +67,6 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
   for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-// Write one 128-element bf16 row (given as 64 packed pairs) into a K-major
-// SW128 tile (two 64-column chunks) at row r.
-__device__ __forceinline__ void store_row_sw128(uint32_t tile, int r, const uint32_t (&pk)[64]) {
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const uint32_t chunk = tile + (u >> 3) * kChunk + r * 128;
-    st_shared_v4(chunk + (((u & 7) ^ (r & 7)) << 4), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-  }
-}
-
 __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -79,16 +75,13 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
   uint8_t* sV = smem + Smem::kV;
   uint8_t* sQ = smem + Smem::kQ;
   uint8_t* sDO = smem + Smem::kDO;
-  uint8_t* sPT = smem + Smem::kPT;
   uint8_t* sDS = smem + Smem::kDS;
-  float* sZl2 = reinterpret_cast<float*>(smem + Smem::kStats);
-  float* sT2 = sZl2 + 128;
-  float* sDv = sZl2 + 256;
+  float* sStats = reinterpret_cast<float*>(smem + Smem::kStats);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::kBars);
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + Smem::kMisc);
   // misc[0] TMEM base, misc[1] abort, misc[2..4] progress (producer, MMA,
-  // compute), misc[5] decision, misc[6] tile head, misc[7] tile query block
-  // (-1 = no more tiles)
+  // compute), misc[5] decision, misc[6..7] head of the tile in Q stage 0/1,
+  // misc[8..9] its query block (kEndMarker = no more tiles)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
   const int tid = threadIdx.x;
@@ -106,8 +99,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
   if (tid == 0) {
     for (int x = 0; x < kNumBars; ++x) {
       uint32_t cnt = 1;
-      if (x == kXFree || x == kPtFull || x == kDsFull) cnt = 128;
-      if (x == kQEmpty || x == kDecEmpty) cnt = 2;
+      if (x == kXRead || x == kPtFull || x == kDsFull || x == kYFree) cnt = 128;
+      if (x == kQEmpty || x == kQEmpty + 1 || x == kDecEmpty) cnt = 2;
       mbar_init(&bars[x], cnt);
     }
     for (int x = 1; x < 16; ++x) misc[x] = 0;
@@ -124,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
   const uint32_t tX = tmem, tY = tmem + 128, tDK = tmem + 256, tDV = tmem + 384;
 
   if (warp == 4) {
-    // ===================== producer =====================
+    // ===================== producer (polling) =====================
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
@@ -135,47 +128,102 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         tma_load_4d(sK + c * kChunk, &p.tm_k, &bars[kKVFull], c * 64, hk, j * kB, b);
         tma_load_4d(sV + c * kChunk, &p.tm_v, &bars[kKVFull], c * 64, hk, j * kB, b);
       }
-      misc[2] = 0x10000u;
-      bool ok = true;
-      int n = 0, kc = 0;
-      for (int g = 0; ok && g < G; ++g) {
-        const int h = p.group_heads[hk][g];
-        const int64_t bh = static_cast<int64_t>(b) * p.Hq + h;
-        for (int i = j; ok && i < p.nQB; ++i) {
-          if (p.fwd_mask && !((p.fwd_mask[(bh * p.nQB + i) * p.mask_words + (j >> 5)] >> (j & 31)) & 1u))
-            continue;
-          if (!mbar_wait(&bars[kQEmpty], (n & 1) ^ 1, abort_flag, p.err, wait_tag(1, kQEmpty, n))) { ok = false; break; }
-          misc[6] = static_cast<uint32_t>(h);
-          misc[7] = static_cast<uint32_t>(i);
-          mbar_expect_tx(&bars[kQFull], kTile + 3 * 512);
-          for (int c = 0; c < 2; ++c)
-            tma_load_4d(sQ + c * kChunk, &p.tm_q, &bars[kQFull], c * 64, h, i * kB, b);
-          const int64_t row0 = bh * p.Npad + static_cast<int64_t>(i) * kB;
-          bulk_load(sZl2, p.zl2 + row0, 512, &bars[kQFull]);
-          bulk_load(sT2, p.t2 + row0, 512, &bars[kQFull]);
-          bulk_load(sDv, p.Dv + row0, 512, &bars[kQFull]);
-          misc[2] = 0x20000u | n;
-          if (!mbar_wait(&bars[kDecFull], n & 1, abort_flag, p.err, wait_tag(1, kDecFull, n))) { ok = false; break; }
-          const uint32_t keep = misc[5];
-          mbar_arrive(&bars[kDecEmpty]);
-          if (keep) {
-            if (!mbar_wait(&bars[kDoEmpty], (kc & 1) ^ 1, abort_flag, p.err, wait_tag(1, kDoEmpty, kc))) { ok = false; break; }
-            mbar_expect_tx(&bars[kDoFull], kTile);
-            for (int c = 0; c < 2; ++c)
-              tma_load_4d(sDO + c * kChunk, &p.tm_do, &bars[kDoFull], c * 64, h, i * kB, b);
-            ++kc;
+      // scan state of the next visited tile (group head g, query block i)
+      int sg = 0, si = j;
+      auto next_tile = [&](int& h_out, int& i_out) -> bool {
+        while (sg < G) {
+          const int h = p.group_heads[hk][sg];
+          const int64_t bh = static_cast<int64_t>(b) * p.Hq + h;
+          while (si < p.nQB) {
+            const int i = si++;
+            if (!p.fwd_mask || ((p.fwd_mask[(bh * p.nQB + i) * p.mask_words + (j >> 5)] >> (j & 31)) & 1u)) {
+              h_out = h;
+              i_out = i;
+              return true;
+            }
           }
-          ++n;
-          misc[2] = 0x30000u | n;
+          ++sg;
+          si = j;
+        }
+        return false;
+      };
+      int n_load = 0, n_dec = 0, kc_load = 0, n_total = -1;   // n_total known once the end marker is loaded
+      int pend_h[2], pend_i[2], pend_n = 0;                    // retained tiles waiting for their dO load
+      // (head, query block) of tile n at [n % 4]: decisions trail the Q loads
+      // by at most three tiles (a tile's Q stage is refilled only after its
+      // decision was published, and the next decision waits for this one to
+      // be read)
+      int info_h[4] = {0, 0, 0, 0}, info_i[4] = {0, 0, 0, 0};
+      uint64_t idle_since = global_timer_ns();
+      bool ok = true;
+      while (ok) {
+        bool progress = false;
+        if (n_total < 0) {
+          const int st = n_load & 1;
+          if (mbar_test(&bars[kQEmpty + st], ((n_load >> 1) & 1) ^ 1)) {
+            int h = 0, i = 0;
+            if (next_tile(h, i)) {
+              info_h[n_load & 3] = h;
+              info_i[n_load & 3] = i;
+              misc[6 + st] = static_cast<uint32_t>(h);
+              misc[8 + st] = static_cast<uint32_t>(i);
+              mbar_expect_tx(&bars[kQFull + st], kTile + 3 * 512);
+              for (int c = 0; c < 2; ++c)
+                tma_load_4d(sQ + st * kTile + c * kChunk, &p.tm_q, &bars[kQFull + st], c * 64, h, i * kB, b);
+              const int64_t row0 = (static_cast<int64_t>(b) * p.Hq + h) * p.Npad + static_cast<int64_t>(i) * kB;
+              float* sst = sStats + st * 384;
+              bulk_load(sst, p.zl2 + row0, 512, &bars[kQFull + st]);
+              bulk_load(sst + 128, p.t2 + row0, 512, &bars[kQFull + st]);
+              bulk_load(sst + 256, p.Dv + row0, 512, &bars[kQFull + st]);
+            } else {
+              misc[8 + st] = kEndMarker;
+              mbar_arrive(&bars[kQFull + st]);
+              n_total = n_load;
+            }
+            ++n_load;
+            progress = true;
+          }
+        }
+        if (n_dec < n_load && (n_total < 0 || n_dec < n_total) && pend_n < 2) {
+          if (mbar_test(&bars[kDecFull], n_dec & 1)) {
+            const uint32_t keep = misc[5];
+            mbar_arrive(&bars[kDecEmpty]);
+            if (keep) {
+              pend_h[pend_n] = info_h[n_dec & 3];
+              pend_i[pend_n] = info_i[n_dec & 3];
+              ++pend_n;
+            }
+            ++n_dec;
+            progress = true;
+          }
+        }
+        if (pend_n > 0 && mbar_test(&bars[kDoEmpty], (kc_load & 1) ^ 1)) {
+          mbar_expect_tx(&bars[kDoFull], kTile);
+          for (int c = 0; c < 2; ++c)
+            tma_load_4d(sDO + c * kChunk, &p.tm_do, &bars[kDoFull], c * 64, pend_h[0], pend_i[0] * kB, b);
+          pend_h[0] = pend_h[1];
+          pend_i[0] = pend_i[1];
+          --pend_n;
+          ++kc_load;
+          progress = true;
+        }
+        misc[2] = (static_cast<uint32_t>(n_load) << 16) | (static_cast<uint32_t>(n_dec) & 0xffff);
+        if (n_total >= 0 && n_dec == n_total && pend_n == 0) break;
+        if (progress) {
+          idle_since = global_timer_ns();
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (global_timer_ns() - idle_since > kWaitLimitNs) {
+          *abort_flag = 1;
+          if (atomicCAS(p.err, 0, kErrTimeout) == 0) {
+            p.err[1] = wait_tag(1, 0xff, n_dec);
+            p.err[2] = static_cast<int>(blockIdx.x);
+            for (int x = 0; x < 3; ++x) p.err[4 + x] = misc[2 + x];
+          }
+          ok = false;
         }
       }
-      // end marker: one more "tile" with query block -1
-      if (ok && mbar_wait(&bars[kQEmpty], (n & 1) ^ 1, abort_flag, p.err, wait_tag(1, kQEmpty, n))) {
-        misc[7] = 0xFFFFFFFFu;
-        mbar_arrive(&bars[kQFull]);
-      } else {
-        drain_pause_ns(50000);
-      }
+      if (!ok) drain_pause_ns(50000);
     }
   } else if (warp == 5) {
     // ===================== tcgen05 issuer =====================
@@ -184,205 +232,116 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       constexpr uint32_t id_kmn = idesc_bf16_f32(128, 128, false, true);   // B MN-major
       constexpr uint32_t id_mnmn = idesc_bf16_f32(128, 128, true, true);   // A, B MN-major
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
-      const uint32_t aPT = smem_u32(sPT), aDS = smem_u32(sDS);
-      bool ok = mbar_wait(&bars[kKVFull], 0, abort_flag, p.err, wait_tag(2, kKVFull, 0));
-      int n = 0, kc = 0;
-      while (ok) {
-        if (!mbar_wait(&bars[kQFull], n & 1, abort_flag, p.err, wait_tag(2, kQFull, n))) { ok = false; break; }
-        if (misc[7] == 0xFFFFFFFFu) break;
-        if (!mbar_wait(&bars[kXFree], (n & 1) ^ 1, abort_flag, p.err, wait_tag(2, kXFree, n))) { ok = false; break; }
-        tc_fence_after();
-        // S^T = K_j Q_i^T (K = d)
+      const uint32_t aDS = smem_u32(sDS);
+      auto issue_s = [&](int n) {
+        const uint32_t q = aQ + (n & 1) * kTile;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
-          umma_bf16_ss(tX, sdesc_sw128(aK + off, 16, 1024), sdesc_sw128(aQ + off, 16, 1024), id_kk, kk > 0);
+          umma_bf16_ss(tX, sdesc_sw128(aK + off, 16, 1024), sdesc_sw128(q + off, 16, 1024), id_kk, kk > 0);
         }
         umma_commit(&bars[kSFull]);
-        misc[3] = 0x10000u | n;
+      };
+      bool ok = mbar_wait(&bars[kKVFull], 0, abort_flag, p.err, wait_tag(2, kKVFull, 0));
+      int n = 0, kc = 0, sk = 0;
+      bool have_next = false;
+      if (ok) ok = mbar_wait(&bars[kQFull], 0, abort_flag, p.err, wait_tag(2, kQFull, 0));
+      if (ok && misc[8] != kEndMarker) {
+        tc_fence_after();
+        issue_s(0);
+        have_next = true;
+      }
+      while (ok && have_next) {
         if (!mbar_wait(&bars[kDecFull], n & 1, abort_flag, p.err, wait_tag(2, kDecFull, n))) { ok = false; break; }
         const uint32_t keep = misc[5];
         mbar_arrive(&bars[kDecEmpty]);
-        if (!keep) {
-          umma_commit(&bars[kQEmpty]);
-          ++n;
-          continue;
-        }
-        if (!mbar_wait(&bars[kDoFull], kc & 1, abort_flag, p.err, wait_tag(2, kDoFull, kc))) { ok = false; break; }
-        if (!mbar_wait(&bars[kPtFull], kc & 1, abort_flag, p.err, wait_tag(2, kPtFull, kc))) { ok = false; break; }
-        tc_fence_after();
-        // dV += P^T dO (K = queries; dO as MN-major B)
+        const int st = n & 1, stn = (n + 1) & 1;
+        if (keep) {
+          if (!mbar_wait(&bars[kPtFull], kc & 1, abort_flag, p.err, wait_tag(2, kPtFull, kc))) { ok = false; break; }
+          if (!mbar_wait(&bars[kDoFull], kc & 1, abort_flag, p.err, wait_tag(2, kDoFull, kc))) { ok = false; break; }
+          tc_fence_after();
+          // dV += P^T dO: A = P^T from TMEM (8 columns per 16 queries), B = dO MN-major
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t offa = (kk >> 2) * kChunk + (kk & 3) * 32;
-          umma_bf16_ss(tDV, sdesc_sw128(aPT + offa, 16, 1024), sdesc_sw128(aDO + kk * 2048, kChunk, 1024), id_kmn,
-                       (kc > 0 || kk > 0) ? 1u : 0u);
-        }
-        // dP^T = V_j dO^T (K = d)
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16_ts(tDV, tX + kk * 8, sdesc_sw128(aDO + kk * 2048, kChunk, 1024), id_kmn,
+                         (kc > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bars[kDvDone]);
+          // dP^T = V_j dO^T into Y once the previous dQ part has left it
+          if (!mbar_wait(&bars[kYFree], (kc & 1) ^ 1, abort_flag, p.err, wait_tag(2, kYFree, kc))) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
-          umma_bf16_ss(tY, sdesc_sw128(aV + off, 16, 1024), sdesc_sw128(aDO + off, 16, 1024), id_kk, kk > 0);
-        }
-        umma_commit(&bars[kDpFull]);
-        umma_commit(&bars[kDoEmpty]);
-        umma_commit(&bars[kPtFree]);
-        misc[3] = 0x20000u | n;
-        if (!mbar_wait(&bars[kDsFull], kc & 1, abort_flag, p.err, wait_tag(2, kDsFull, kc))) { ok = false; break; }
-        tc_fence_after();
-        // dK += dS^T Q_i (K = queries; Q as MN-major B)
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kChunk + (kk & 3) * 32;
+            umma_bf16_ss(tY, sdesc_sw128(aV + off, 16, 1024), sdesc_sw128(aDO + off, 16, 1024), id_kk, kk > 0);
+          }
+          umma_commit(&bars[kDpFull]);
+          umma_commit(&bars[kDoEmpty]);
+          // S^T of the next tile into X once dV has read P^T from it
+          if (!mbar_wait(&bars[kQFull + stn], ((n + 1) >> 1) & 1, abort_flag, p.err, wait_tag(2, kQFull + stn, n + 1))) { ok = false; break; }
+          have_next = misc[8 + stn] != kEndMarker;
+          if (have_next) {
+            if (!mbar_wait(&bars[kDvDone], kc & 1, abort_flag, p.err, wait_tag(2, kDvDone, kc))) { ok = false; break; }
+            tc_fence_after();
+            issue_s(n + 1);
+          }
+          // dK += dS^T Q_i and the dQ part = dS K_j into Y
+          if (!mbar_wait(&bars[kDsFull], kc & 1, abort_flag, p.err, wait_tag(2, kDsFull, kc))) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t q = aQ + st * kTile;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t offa = (kk >> 2) * kChunk + (kk & 3) * 32;
-          umma_bf16_ss(tDK, sdesc_sw128(aDS + offa, 16, 1024), sdesc_sw128(aQ + kk * 2048, kChunk, 1024), id_kmn,
-                       (kc > 0 || kk > 0) ? 1u : 0u);
-        }
-        // dQ part = dS K_j (K = keys; dS^T tile read as MN-major A, K_j as MN-major B)
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t offa = (kk >> 2) * kChunk + (kk & 3) * 32;
+            umma_bf16_ss(tDK, sdesc_sw128(aDS + offa, 16, 1024), sdesc_sw128(q + kk * 2048, kChunk, 1024), id_kmn,
+                         (kc > 0 || kk > 0) ? 1u : 0u);
+          }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          umma_bf16_ss(tX, sdesc_sw128(aDS + kk * 2048, kChunk, 1024), sdesc_sw128(aK + kk * 2048, kChunk, 1024),
-                       id_mnmn, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16_ss(tY, sdesc_sw128(aDS + kk * 2048, kChunk, 1024), sdesc_sw128(aK + kk * 2048, kChunk, 1024),
+                         id_mnmn, kk > 0);
+          umma_commit(&bars[kDqFull]);
+          umma_commit(&bars[kQEmpty + st]);
+          ++kc;
+        } else {
+          umma_commit(&bars[kQEmpty + st]);
+          if (!mbar_wait(&bars[kQFull + stn], ((n + 1) >> 1) & 1, abort_flag, p.err, wait_tag(2, kQFull + stn, n + 1))) { ok = false; break; }
+          have_next = misc[8 + stn] != kEndMarker;
+          if (have_next) {
+            if (!mbar_wait(&bars[kXRead], sk & 1, abort_flag, p.err, wait_tag(2, kXRead, sk))) { ok = false; break; }
+            tc_fence_after();
+            issue_s(n + 1);
+          }
+          ++sk;
         }
-        umma_commit(&bars[kDqFull]);
-        umma_commit(&bars[kQEmpty]);
-        umma_commit(&bars[kDsFree]);
-        misc[3] = 0x30000u | n;
-        ++kc;
+        misc[3] = (static_cast<uint32_t>(n) << 16) | (static_cast<uint32_t>(kc) & 0xffff);
         ++n;
       }
+      // every MMA issued above must have finished before TMEM is read or freed
       umma_commit(&bars[kDone]);
       mbar_wait(&bars[kDone], 0, abort_flag, p.err, wait_tag(2, kDone, 0));
     }
   } else {
     // ===================== compute warpgroup =====================
-    const int t = tid;                          // key row (S^T, dK, dV) / query row (dQ part)
+    const int t = tid;                          // key row (S^T, P^T, dP^T, dS^T) / query row (dQ part)
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t aPT = smem_u32(sPT), aDS = smem_u32(sDS);
-    int n = 0, kc = 0, visited = 0, kept = 0;
+    const uint32_t aDS = smem_u32(sDS);
+    int n = 0, kc = 0, sk = 0, visited = 0, kept = 0;
     int64_t slots = 0;
-    while (true) {
-      const bool okq = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull], n & 1, abort_flag, p.err, wait_tag(0, kQFull, n)));
-      const uint32_t qi = misc[7];
-      if (bar_or(1, 128, !okq || *abort_flag != 0) || qi == 0xFFFFFFFFu) break;
-      const int i = static_cast<int>(qi);
-      const int h = static_cast<int>(misc[6]);
-      uint32_t sr[4][32];
-      const bool oks = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], n & 1, abort_flag, p.err, wait_tag(0, kSFull, n)));
-      if (oks) {
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tX + lane_addr + c * 32, sr[c]);
-          tmem_ld_wait(sr[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int x = 0; x < 32; ++x) sr[c][x] = 0u;
-      }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
-      // legal entries: query column c >= key row t on the diagonal tile; padded
-      // query rows carry t2 = zl2 = +inf and never count
-      const int lim = (i == j) ? t : 0;         // first legal column
-      bool vote = false;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int col = c * 32 + x;
-          const float s2 = __uint_as_float(sr[c][x]) * kLog2e;
-          vote |= (col >= lim) && (s2 >= sT2[col]);
-        }
-      const bool keep = bar_or(1, 128, vote);
-      misc[4] = 0x10000u | n;
-      if (tid == 0) {
-        if (mbar_wait(&bars[kDecEmpty], (n & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty, n))) {
-          misc[5] = keep ? 1u : 0u;
-          mbar_arrive(&bars[kDecFull]);
-        }
-        ++visited;
-        if (keep) {
-          ++kept;
-          slots += static_cast<int64_t>(kB) * min(kB, p.N - i * kB);
-          if (p.bwd_mask)
-            atomicOr(&p.bwd_mask[((static_cast<int64_t>(b) * p.Hq + h) * p.nQB + i) * p.mask_words + (j >> 5)],
-                     1u << (j & 31));
-        }
-      }
-      if (!keep) {
-        tc_fence_before();
-        mbar_arrive(&bars[kXFree]);
-        if (tid == 0) mbar_arrive(&bars[kQEmpty]);
-        ++n;
-        continue;
-      }
+    bool pending = false;                       // a dQ part waits in Y
+    int pend_h = 0, pend_i = 0;
 
-      // P^T = exp2(S^T log2e - z log2e) on legal entries (fp32 kept for dS)
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int col = c * 32 + x;
-          const float pv = (col >= lim) ? ex2_approx(fmaf(__uint_as_float(sr[c][x]), kLog2e, -sZl2[col])) : 0.0f;
-          sr[c][x] = __float_as_uint(pv);
-        }
-      mbar_wait(&bars[kPtFree], (kc & 1) ^ 1, abort_flag, p.err, wait_tag(0, kPtFree, kc));
-      {
-        uint32_t pk[64];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int x = 0; x < 32; x += 2)
-            pk[c * 16 + (x >> 1)] = pack_bf16x2(__uint_as_float(sr[c][x]), __uint_as_float(sr[c][x + 1]));
-        store_row_sw128(aPT, t, pk);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&bars[kPtFull]);
-
-      // dS^T = P^T (dP^T - D)
-      const bool okd = __all_sync(0xffffffffu, mbar_wait(&bars[kDpFull], kc & 1, abort_flag, p.err, wait_tag(0, kDpFull, kc)));
-      mbar_wait(&bars[kDsFree], (kc & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDsFree, kc));
-      {
-        uint32_t pk[64];
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t dp[32];
-          if (okd) {
-            tmem_ld32(tY + lane_addr + c * 32, dp);
-            tmem_ld_wait(dp);
-          } else {
-#pragma unroll
-            for (int x = 0; x < 32; ++x) dp[x] = 0u;
-          }
-          reg_fence(dp);
-#pragma unroll
-          for (int x = 0; x < 32; x += 2) {
-            const int col = c * 32 + x;
-            const float d0 = __uint_as_float(sr[c][x]) * (__uint_as_float(dp[x]) - sDv[col]);
-            const float d1 = __uint_as_float(sr[c][x + 1]) * (__uint_as_float(dp[x + 1]) - sDv[col + 1]);
-            pk[c * 16 + (x >> 1)] = pack_bf16x2(d0, d1);
-          }
-        }
-        store_row_sw128(aDS, t, pk);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars[kDsFull]);
-      if (tid == 0) mbar_arrive(&bars[kQEmpty]);
-
-      // dQ part (query row t) -> fp32 staging in the P^T tile -> bulk add into dQ_acc
-      const bool okq2 = __all_sync(0xffffffffu, mbar_wait(&bars[kDqFull], kc & 1, abort_flag, p.err, wait_tag(0, kDqFull, kc)));
+    // dQ part of the previous retained tile: TMEM -> fp32 staging in the dS^T
+    // tile -> bulk add into the blocked dQ accumulator; frees Y
+    auto drain = [&]() {
+      const bool okq = __all_sync(0xffffffffu, mbar_wait(&bars[kDqFull], (kc - 1) & 1, abort_flag, p.err,
+                                                          wait_tag(0, kDqFull, kc - 1)));
       tc_fence_after();
-      float* stage = reinterpret_cast<float*>(sPT);
-      float* dst = p.dq_acc + (((static_cast<int64_t>(b) * p.Hq + h) * p.nQB + i) * 4) * (kB * 32);
+      float* stage = reinterpret_cast<float*>(sDS);
+      float* dst = p.dq_acc + (((static_cast<int64_t>(b) * p.Hq + pend_h) * p.nQB + pend_i) * 4) * (kB * 32);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t dq[32];
-        if (okq2) {
-          tmem_ld32(tX + lane_addr + c * 32, dq);
+        if (okq) {
+          tmem_ld32(tY + lane_addr + c * 32, dq);
           tmem_ld_wait(dq);
         } else {
 #pragma unroll
@@ -390,8 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         }
         reg_fence(dq);
         if (c >= 2) {
-          // staging half c & 1 is reused: its previous bulk add must have read it
-          if (tid == 0) bulk_wait_read<1>();
+          if (tid == 0) bulk_wait_read<1>();    // staging half c & 1 was read by its bulk add
           named_bar_sync(1, 128);
         }
         float* row = stage + (c & 1) * (kB * 32) + t * 32;
@@ -408,13 +366,145 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         }
       }
       tc_fence_before();
-      mbar_arrive(&bars[kXFree]);
-      // the P^T tile is free again once the bulk adds have read the staging
+      mbar_arrive(&bars[kYFree]);
+      // the dS^T tile is rewritten next: the bulk adds must have read it
       if (tid == 0) bulk_wait_read<0>();
       named_bar_sync(1, 128);
+      pending = false;
+    };
+
+    while (true) {
+      const int st = n & 1;
+      const bool okq = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull + st], (n >> 1) & 1, abort_flag, p.err,
+                                                         wait_tag(0, kQFull + st, n)));
+      const uint32_t qi = misc[8 + st];
+      if (bar_or(1, 128, !okq || *abort_flag != 0) || qi == kEndMarker) break;
+      const int i = static_cast<int>(qi);
+      const int h = static_cast<int>(misc[6 + st]);
+      const float* sZl2 = sStats + st * 384;
+      const float* sThr = sZl2 + 128;
+      const float* sDv = sZl2 + 256;
+      // test pass: stream S^T in 32-column chunks (legal entries: query column
+      // c >= key row t on the diagonal tile; padded query rows carry an
+      // infinite threshold and never count)
+      const bool oks = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], n & 1, abort_flag, p.err, wait_tag(0, kSFull, n)));
+      const int lim = (i == j) ? t : 0;
+      bool vote = false;
+      if (oks) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sr[32];
+          tmem_ld32(tX + lane_addr + c * 32, sr);
+          tmem_ld_wait(sr);
+          reg_fence(sr);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const int col = c * 32 + x;
+            vote |= (col >= lim) && (__uint_as_float(sr[x]) >= sThr[col]);
+          }
+        }
+      }
+      const bool keep = bar_or(1, 128, vote);
+      if (tid == 0) {
+        misc[4] = (static_cast<uint32_t>(n) << 16) | (static_cast<uint32_t>(kc) & 0xffff);
+        if (mbar_wait(&bars[kDecEmpty], (n & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty, n))) {
+          misc[5] = keep ? 1u : 0u;
+          mbar_arrive(&bars[kDecFull]);
+        }
+        ++visited;
+        if (keep) {
+          ++kept;
+          slots += static_cast<int64_t>(kB) * min(kB, p.N - i * kB);
+          if (p.bwd_mask)
+            atomicOr(&p.bwd_mask[((static_cast<int64_t>(b) * p.Hq + h) * p.nQB + i) * p.mask_words + (j >> 5)],
+                     1u << (j & 31));
+        }
+      }
+      if (!keep) {
+        tc_fence_before();
+        mbar_arrive(&bars[kXRead]);
+        if (tid == 0) mbar_arrive(&bars[kQEmpty + st]);
+        ++sk;
+        ++n;
+        if (pending) drain();
+        continue;
+      }
+
+      // P^T = exp2(S^T log2e - z log2e) on legal entries, as bf16 pairs: kept
+      // in registers for dS and written over S^T in X for the dV MMA. Chunk c
+      // of P^T (16 columns) lands on columns of S^T chunks already read.
+      uint32_t pp[64];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[32];
+        if (oks) {
+          tmem_ld32(tX + lane_addr + c * 32, sr);
+          tmem_ld_wait(sr);
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) sr[x] = 0u;
+        }
+        reg_fence(sr);
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const int col = c * 32 + x;
+          const float p0 = (col >= lim) ? ex2_approx(fmaf(__uint_as_float(sr[x]), kLog2e, -sZl2[col])) : 0.0f;
+          const float p1 = (col + 1 >= lim) ? ex2_approx(fmaf(__uint_as_float(sr[x + 1]), kLog2e, -sZl2[col + 1])) : 0.0f;
+          pp[c * 16 + (x >> 1)] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tX + lane_addr + c * 16, &pp[c * 16]);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[kPtFull]);
+
+      if (pending) drain();
+
+      // dS^T = P^T (dP^T - D) -> bf16 into the dS^T tile
+      const bool okd = __all_sync(0xffffffffu, mbar_wait(&bars[kDpFull], kc & 1, abort_flag, p.err, wait_tag(0, kDpFull, kc)));
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t dp[32];
+        if (okd) {
+          tmem_ld32(tY + lane_addr + c * 32, dp);
+          tmem_ld_wait(dp);
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) dp[x] = 0u;
+        }
+        reg_fence(dp);
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const int col = c * 32 + x;
+          const uint32_t w = pp[c * 16 + (x >> 1)];
+          const float p0 = __uint_as_float(w << 16);
+          const float p1 = __uint_as_float(w & 0xFFFF0000u);
+          const float d0 = p0 * (__uint_as_float(dp[x]) - sDv[col]);
+          const float d1 = p1 * (__uint_as_float(dp[x + 1]) - sDv[col + 1]);
+          pk[x >> 1] = pack_bf16x2(d0, d1);
+        }
+        // queries [32c, 32c+32): chunk c / 2, 16-byte units (c & 1) * 4 + 0..3
+        const uint32_t rowb = aDS + (c >> 1) * kChunk + t * 128;
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const uint32_t u = (c & 1) * 4 + u4;
+          st_shared_v4(rowb + ((u ^ (t & 7)) << 4), pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars[kDsFull]);
+      if (tid == 0) mbar_arrive(&bars[kQEmpty + st]);
+      pending = true;
+      pend_h = h;
+      pend_i = i;
       ++kc;
       ++n;
     }
+    if (pending && !*abort_flag) drain();
 
     // dK_j, dV_j (key row t) -> bf16
     if (tid == 0) bulk_wait_all<0>();
@@ -422,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
     const int krow = j * kB + t;
     if (okdone && !*abort_flag) {
       tc_fence_after();
-      const bool any_kept = kc > 0;           // dK/dV TMEM untouched when nothing was retained
+      const bool any_kept = kc > 0;            // dK/dV TMEM untouched when nothing was retained
       __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(p.dk) + b * p.dk_sb + static_cast<int64_t>(krow) * p.dk_sn + hk * p.dk_sh;
       __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(p.dv) + b * p.dv_sb + static_cast<int64_t>(krow) * p.dv_sn + hk * p.dv_sh;
 #pragma unroll
@@ -462,7 +552,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
   }
 }
 
-// D = rowsum(dO o O), zl2 = z log2e, t2 = (z + log tau - log(q + 1)) log2e,
+// D = rowsum(dO o O), zl2 = z log2e, t2 = z + log tau - log(q + 1) (the
+// score a legal entry must reach to retain the tile, natural log units),
 // padded rows: zl2 = t2 = +inf, D = 0; zero the block's dQ accumulator.
 __global__ void __launch_bounds__(128) mala_bwd_pre_kernel(const __grid_constant__ BwdAuxParams p) {
   const int blk = blockIdx.x;                  // (b, h, i)
@@ -494,7 +585,7 @@ __global__ void __launch_bounds__(128) mala_bwd_pre_kernel(const __grid_constant
     const float z = p.lse[static_cast<int64_t>(bh) * p.N + q];
     p.Dv[row] = acc;
     p.zl2[row] = z * kLog2e;
-    p.t2[row] = (z + p.log_tau - logf(static_cast<float>(q + 1))) * kLog2e;
+    p.t2[row] = z + p.log_tau - logf(static_cast<float>(q + 1));
   } else {
     p.Dv[row] = 0.0f;
     p.zl2[row] = INFINITY;

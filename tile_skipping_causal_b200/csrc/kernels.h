@@ -79,7 +79,7 @@ size_t decode_smem_bytes();
 struct BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;   // 4-D maps, box {64, 1, 128, 1}, 128B swizzle
   const float* zl2;        // [B, Hq, Npad] z log2e
-  const float* t2;         // [B, Hq, Npad] (z + log tau - log L_q) log2e
+  const float* t2;         // [B, Hq, Npad] z + log tau - log L_q (natural log)
   const float* Dv;         // [B, Hq, Npad] rowsum(dO o O)
   float* dq_acc;           // [B, Hq, nQB, 4, 128, 32] fp32
   void* dk;
