@@ -9,7 +9,7 @@
 // (q, k) s_qk - z_q < log tau - log L_q. A retained tile loads dO_i and runs
 //   P^T = exp(S^T - z), dV += P^T dO, dP^T = V dO^T, dS^T = P^T (dP^T - D),
 //   dK += dS^T Q, dQ_i += dS K
-// with dQ accumulated in fp32 by bulk reduce-add into a blocked workspace.
+// with dQ accumulated in fp32 by vector reductions into a blocked workspace.
 //
 // Roles (192 threads): warps 0-3 compute (thread t owns key row t for
 // S^T, P^T, dP^T, dS^T and query row t for the dQ part), warp 4 TMA
@@ -18,9 +18,8 @@
 // TMEM: X = cols [0,128): S^T(n), then P^T(n) as packed bf16 in [0,64),
 // read by the dV MMA straight from TMEM; Y = [128,256): dP^T(n), then the
 // tile's dQ part; dK = [256,384); dV = [384,512).
-// Shared memory: K_j, V_j, two Q_i stages (with their row statistics), dO_i,
-// and the dS^T tile, which doubles as the fp32 staging buffer of the dQ
-// reduction once dK and dQ have consumed it.
+// Shared memory: K_j, V_j, two Q_i stages (with their row statistics), dO_i
+// and the dS^T tile.
 //
 // Issue order of the tensor pipe for a retained tile n:
 //   dV(n), dP^T(n) -> Y, S^T(n+1) -> X, dK(n), dQ(n) -> Y
@@ -329,47 +328,43 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
     bool pending = false;                       // a dQ part waits in Y
     int pend_h = 0, pend_i = 0;
 
-    // dQ part of the previous retained tile: TMEM -> fp32 staging in the dS^T
-    // tile -> bulk add into the blocked dQ accumulator; frees Y
+    // dQ part of the previous retained tile (query row t): TMEM -> registers
+    // -> vector fp32 reductions into the accumulator, whose layout
+    // [.., 32 column quads, 128 rows, 4] makes each warp instruction cover
+    // 512 contiguous bytes; frees Y
     auto drain = [&]() {
       const bool okq = __all_sync(0xffffffffu, mbar_wait(&bars[kDqFull], (kc - 1) & 1, abort_flag, p.err,
                                                           wait_tag(0, kDqFull, kc - 1)));
       tc_fence_after();
-      float* stage = reinterpret_cast<float*>(sDS);
-      float* dst = p.dq_acc + (((static_cast<int64_t>(b) * p.Hq + pend_h) * p.nQB + pend_i) * 4) * (kB * 32);
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t dq[32];
+      float* dst = p.dq_acc + ((static_cast<int64_t>(b) * p.Hq + pend_h) * p.nQB + pend_i) * (kB * kD) + t * 4;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t q0[32], q1[32];
         if (okq) {
-          tmem_ld32(tY + lane_addr + c * 32, dq);
-          tmem_ld_wait(dq);
+          tmem_ld32(tY + lane_addr + half * 64, q0);
+          tmem_ld32(tY + lane_addr + half * 64 + 32, q1);
+          tmem_ld_wait(q0);
         } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) dq[x] = 0u;
+          for (int x = 0; x < 32; ++x) q0[x] = q1[x] = 0u;
         }
-        reg_fence(dq);
-        if (c >= 2) {
-          if (tid == 0) bulk_wait_read<1>();    // staging half c & 1 was read by its bulk add
-          named_bar_sync(1, 128);
-        }
-        float* row = stage + (c & 1) * (kB * 32) + t * 32;
+        reg_fence(q0);
+        reg_fence(q1);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int u = (k + t) & 7;             // rotate to spread banks
-          *reinterpret_cast<uint4*>(row + 4 * u) = make_uint4(dq[4 * u], dq[4 * u + 1], dq[4 * u + 2], dq[4 * u + 3]);
+        for (int u = 0; u < 8; ++u) {
+          const int quad = half * 16 + u;
+          red_add_v4_f32(dst + quad * (kB * 4), __uint_as_float(q0[4 * u]), __uint_as_float(q0[4 * u + 1]),
+                         __uint_as_float(q0[4 * u + 2]), __uint_as_float(q0[4 * u + 3]));
         }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (tid == 0) {
-          bulk_reduce_add_f32(dst + c * (kB * 32), stage + (c & 1) * (kB * 32), kB * 32 * 4);
-          bulk_commit_group();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int quad = half * 16 + 8 + u;
+          red_add_v4_f32(dst + quad * (kB * 4), __uint_as_float(q1[4 * u]), __uint_as_float(q1[4 * u + 1]),
+                         __uint_as_float(q1[4 * u + 2]), __uint_as_float(q1[4 * u + 3]));
         }
       }
       tc_fence_before();
       mbar_arrive(&bars[kYFree]);
-      // the dS^T tile is rewritten next: the bulk adds must have read it
-      if (tid == 0) bulk_wait_read<0>();
-      named_bar_sync(1, 128);
       pending = false;
     };
 
@@ -384,27 +379,33 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       const float* sZl2 = sStats + st * 384;
       const float* sThr = sZl2 + 128;
       const float* sDv = sZl2 + 256;
-      // test pass: stream S^T in 32-column chunks (legal entries: query column
-      // c >= key row t on the diagonal tile; padded query rows carry an
-      // infinite threshold and never count)
+      // test pass over S^T (one batched TMEM load of the row). Legal entries:
+      // query column c >= key row t on the diagonal tile; padded query rows
+      // carry an infinite threshold and never count
       const bool oks = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], n & 1, abort_flag, p.err, wait_tag(0, kSFull, n)));
       const int lim = (i == j) ? t : 0;
       bool vote = false;
+      uint32_t sr[4][32];
       if (oks) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sr[32];
-          tmem_ld32(tX + lane_addr + c * 32, sr);
-          tmem_ld_wait(sr);
-          reg_fence(sr);
+        for (int c = 0; c < 4; ++c) tmem_ld32(tX + lane_addr + c * 32, sr[c]);
+        tmem_ld_wait(sr[0]);
+      } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const int col = c * 32 + x;
-            vote |= (col >= lim) && (__uint_as_float(sr[x]) >= sThr[col]);
-          }
-        }
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int x = 0; x < 32; ++x) sr[c][x] = 0u;
       }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const int col = c * 32 + x;
+          vote |= (col >= lim) && (__uint_as_float(sr[c][x]) >= sThr[col]);
+        }
       const bool keep = bar_or(1, 128, vote);
       if (tid == 0) {
         misc[4] = (static_cast<uint32_t>(n) << 16) | (static_cast<uint32_t>(kc) & 0xffff);
@@ -432,25 +433,16 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       }
 
       // P^T = exp2(S^T log2e - z log2e) on legal entries, as bf16 pairs: kept
-      // in registers for dS and written over S^T in X for the dV MMA. Chunk c
-      // of P^T (16 columns) lands on columns of S^T chunks already read.
+      // in registers for dS and written over S^T in X for the dV MMA (chunk c
+      // of P^T, 16 columns, lands on S^T columns already read)
       uint32_t pp[64];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t sr[32];
-        if (oks) {
-          tmem_ld32(tX + lane_addr + c * 32, sr);
-          tmem_ld_wait(sr);
-        } else {
-#pragma unroll
-          for (int x = 0; x < 32; ++x) sr[x] = 0u;
-        }
-        reg_fence(sr);
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
           const int col = c * 32 + x;
-          const float p0 = (col >= lim) ? ex2_approx(fmaf(__uint_as_float(sr[x]), kLog2e, -sZl2[col])) : 0.0f;
-          const float p1 = (col + 1 >= lim) ? ex2_approx(fmaf(__uint_as_float(sr[x + 1]), kLog2e, -sZl2[col + 1])) : 0.0f;
+          const float p0 = (col >= lim) ? ex2_approx(fmaf(__uint_as_float(sr[c][x]), kLog2e, -sZl2[col])) : 0.0f;
+          const float p1 = (col + 1 >= lim) ? ex2_approx(fmaf(__uint_as_float(sr[c][x + 1]), kLog2e, -sZl2[col + 1])) : 0.0f;
           pp[c * 16 + (x >> 1)] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tX + lane_addr + c * 16, &pp[c * 16]);
@@ -465,33 +457,39 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       const bool okd = __all_sync(0xffffffffu, mbar_wait(&bars[kDpFull], kc & 1, abort_flag, p.err, wait_tag(0, kDpFull, kc)));
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t dp[32];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t dp[2][32];
         if (okd) {
-          tmem_ld32(tY + lane_addr + c * 32, dp);
-          tmem_ld_wait(dp);
+          tmem_ld32(tY + lane_addr + half * 64, dp[0]);
+          tmem_ld32(tY + lane_addr + half * 64 + 32, dp[1]);
+          tmem_ld_wait(dp[0]);
         } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) dp[x] = 0u;
+          for (int x = 0; x < 32; ++x) dp[0][x] = dp[1][x] = 0u;
         }
-        reg_fence(dp);
-        uint32_t pk[16];
+        reg_fence(dp[0]);
+        reg_fence(dp[1]);
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          const int col = c * 32 + x;
-          const uint32_t w = pp[c * 16 + (x >> 1)];
-          const float p0 = __uint_as_float(w << 16);
-          const float p1 = __uint_as_float(w & 0xFFFF0000u);
-          const float d0 = p0 * (__uint_as_float(dp[x]) - sDv[col]);
-          const float d1 = p1 * (__uint_as_float(dp[x + 1]) - sDv[col + 1]);
-          pk[x >> 1] = pack_bf16x2(d0, d1);
-        }
-        // queries [32c, 32c+32): chunk c / 2, 16-byte units (c & 1) * 4 + 0..3
-        const uint32_t rowb = aDS + (c >> 1) * kChunk + t * 128;
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = half * 2 + cc;
+          uint32_t pk[16];
 #pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
-          const uint32_t u = (c & 1) * 4 + u4;
-          st_shared_v4(rowb + ((u ^ (t & 7)) << 4), pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
+          for (int x = 0; x < 32; x += 2) {
+            const int col = c * 32 + x;
+            const uint32_t w = pp[c * 16 + (x >> 1)];
+            const float p0 = __uint_as_float(w << 16);
+            const float p1 = __uint_as_float(w & 0xFFFF0000u);
+            const float d0 = p0 * (__uint_as_float(dp[cc][x]) - sDv[col]);
+            const float d1 = p1 * (__uint_as_float(dp[cc][x + 1]) - sDv[col + 1]);
+            pk[x >> 1] = pack_bf16x2(d0, d1);
+          }
+          // queries [32c, 32c+32): chunk c / 2, 16-byte units (c & 1) * 4 + 0..3
+          const uint32_t rowb = aDS + (c >> 1) * kChunk + t * 128;
+#pragma unroll
+          for (int u4 = 0; u4 < 4; ++u4) {
+            const uint32_t u = (c & 1) * 4 + u4;
+            st_shared_v4(rowb + ((u ^ (t & 7)) << 4), pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
+          }
         }
       }
       fence_proxy_async_smem();
@@ -507,7 +505,6 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
     if (pending && !*abort_flag) drain();
 
     // dK_j, dV_j (key row t) -> bf16
-    if (tid == 0) bulk_wait_all<0>();
     const bool okdone = __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0, abort_flag, p.err, wait_tag(0, kDone, 0)));
     const int krow = j * kB + t;
     if (okdone && !*abort_flag) {
@@ -596,7 +593,7 @@ __global__ void __launch_bounds__(128) mala_bwd_pre_kernel(const __grid_constant
 }
 
 // dQ (bf16, [B, N, Hq, d]) from the blocked fp32 accumulator
-// [B, Hq, nQB, 4 column groups, 128 rows, 32].
+// [B, Hq, nQB, 32 column quads, 128 rows, 4].
 __global__ void __launch_bounds__(128) mala_bwd_dq_kernel(const __grid_constant__ BwdAuxParams p) {
   const int blk = blockIdx.x;
   const int i = blk % p.nQB;
@@ -605,21 +602,15 @@ __global__ void __launch_bounds__(128) mala_bwd_dq_kernel(const __grid_constant_
   const int t = threadIdx.x;
   const int q = i * kB + t;
   if (q >= p.N) return;
-  const float* src = p.dq_acc + (static_cast<int64_t>(bh) * p.nQB + i) * (kB * kD);
+  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + (static_cast<int64_t>(bh) * p.nQB + i) * (kB * kD)) + t;
   __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.dq) + b * p.dq_sb + static_cast<int64_t>(q) * p.dq_sn + h * p.dq_sh;
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const float4* s4 = reinterpret_cast<const float4*>(src + (c * kB + t) * 32);
-    uint32_t pk[16];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const float4 v = s4[u];
-      pk[2 * u] = pack_bf16x2(v.x, v.y);
-      pk[2 * u + 1] = pack_bf16x2(v.z, v.w);
-    }
-    uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) d4[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+  for (int u = 0; u < 16; ++u) {
+    const float4 v0 = src[(2 * u) * kB];
+    const float4 v1 = src[(2 * u + 1) * kB];
+    d4[u] = make_uint4(pack_bf16x2(v0.x, v0.y), pack_bf16x2(v0.z, v0.w), pack_bf16x2(v1.x, v1.y),
+                       pack_bf16x2(v1.z, v1.w));
   }
 }
 

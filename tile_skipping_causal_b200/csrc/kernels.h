@@ -81,7 +81,7 @@ struct BwdParams {
   const float* zl2;        // [B, Hq, Npad] z log2e
   const float* t2;         // [B, Hq, Npad] z + log tau - log L_q (natural log)
   const float* Dv;         // [B, Hq, Npad] rowsum(dO o O)
-  float* dq_acc;           // [B, Hq, nQB, 4, 128, 32] fp32
+  float* dq_acc;           // [B, Hq, nQB, 32 column quads, 128 rows, 4] fp32
   void* dk;
   void* dv;
   const uint32_t* fwd_mask;  // [B, Hq, nQB, mask_words] or NULL (visit every legal tile)
