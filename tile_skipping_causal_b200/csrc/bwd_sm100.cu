@@ -11,10 +11,11 @@
 //   dK += dS^T Q, dQ_i += dS K
 // with dQ accumulated in fp32 by vector reductions into a blocked workspace.
 //
-// Roles (192 threads): warps 0-3 compute (thread t owns key row t for
-// S^T, P^T, dP^T, dS^T and query row t for the dQ part), warp 4 TMA
-// producer (polling: Q of the next tiles and dO of retained tiles), warp 5
-// tcgen05 issuer.
+// Roles (320 threads): warps 0-7 compute in two warpgroups that split the
+// 128 query columns of a tile (lane t of TMEM is key row t for S^T, P^T,
+// dP^T, dS^T and query row t for the dQ part), warp 8 TMA producer
+// (polling: Q of the next tiles and dO of retained tiles), warp 9 tcgen05
+// issuer.
 // TMEM: X = cols [0,128): S^T(n), then P^T(n) as packed bf16 in [0,64),
 // read by the dV MMA straight from TMEM; Y = [128,256): dP^T(n), then the
 // tile's dQ part; dK = [256,384); dV = [384,512).
@@ -35,7 +36,7 @@ namespace {
 
 constexpr int kB = 128;                       // B_q = B_k
 constexpr int kD = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kTile = kB * kD * 2;       // 32 KB bf16 tile
 constexpr uint32_t kChunk = 16384;            // one 64-column swizzle chunk of 128 rows
 constexpr float kLog2e = 1.4426950408889634f;
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
   if (tid == 0) {
     for (int x = 0; x < kNumBars; ++x) {
       uint32_t cnt = 1;
-      if (x == kXRead || x == kPtFull || x == kDsFull || x == kYFree) cnt = 128;
+      if (x == kXRead || x == kPtFull || x == kDsFull || x == kYFree) cnt = 256;
       if (x == kQEmpty || x == kQEmpty + 1 || x == kDecEmpty) cnt = 2;
       mbar_init(&bars[x], cnt);
     }
@@ -115,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
   const uint32_t tmem = misc[0];
   const uint32_t tX = tmem, tY = tmem + 128, tDK = tmem + 256, tDV = tmem + 384;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ===================== producer (polling) =====================
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       }
       if (!ok) drain_pause_ns(50000);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ===================== tcgen05 issuer =====================
     if (lane == 0) {
       constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);   // A, B K-major
@@ -319,52 +320,50 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       mbar_wait(&bars[kDone], 0, abort_flag, p.err, wait_tag(2, kDone, 0));
     }
   } else {
-    // ===================== compute warpgroup =====================
-    const int t = tid;                          // key row (S^T, P^T, dP^T, dS^T) / query row (dQ part)
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    // ===================== compute warpgroups =====================
+    // warps 0-3 take query columns [0, 64), warps 4-7 columns [64, 128);
+    // (warp, lane) owns TMEM lane r = 32 (warp % 4) + lane: key row r of
+    // S^T, P^T, dP^T, dS^T and query row r of the dQ part
+    const int r = ((warp & 3) << 5) | lane;
+    const int half = warp >> 2;
+    const int c0 = half * 64;                   // first query column of this half
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t aDS = smem_u32(sDS);
     int n = 0, kc = 0, sk = 0, visited = 0, kept = 0;
     int64_t slots = 0;
     bool pending = false;                       // a dQ part waits in Y
     int pend_h = 0, pend_i = 0;
 
-    // dQ part of the previous retained tile (query row t): TMEM -> registers
-    // -> vector fp32 reductions into the accumulator, whose layout
-    // [.., 32 column quads, 128 rows, 4] makes each warp instruction cover
-    // 512 contiguous bytes; frees Y
+    // dQ part of the previous retained tile (query row r, this half's 64
+    // columns): TMEM -> registers -> vector fp32 reductions into the
+    // accumulator, whose layout [.., 32 column quads, 128 rows, 4] makes each
+    // warp instruction cover 512 contiguous bytes; frees Y
     auto drain = [&]() {
       const bool okq = __all_sync(0xffffffffu, mbar_wait(&bars[kDqFull], (kc - 1) & 1, abort_flag, p.err,
                                                           wait_tag(0, kDqFull, kc - 1)));
-      tc_fence_after();
-      float* dst = p.dq_acc + ((static_cast<int64_t>(b) * p.Hq + pend_h) * p.nQB + pend_i) * (kB * kD) + t * 4;
+      uint32_t q0[32], q1[32];
+      if (okq) {
+        tc_fence_after();
+        tmem_ld32(tY + lane_addr + c0, q0);
+        tmem_ld32(tY + lane_addr + c0 + 32, q1);
+        tmem_ld_wait(q0);
+      } else {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t q0[32], q1[32];
-        if (okq) {
-          tmem_ld32(tY + lane_addr + half * 64, q0);
-          tmem_ld32(tY + lane_addr + half * 64 + 32, q1);
-          tmem_ld_wait(q0);
-        } else {
-#pragma unroll
-          for (int x = 0; x < 32; ++x) q0[x] = q1[x] = 0u;
-        }
-        reg_fence(q0);
-        reg_fence(q1);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int quad = half * 16 + u;
-          red_add_v4_f32(dst + quad * (kB * 4), __uint_as_float(q0[4 * u]), __uint_as_float(q0[4 * u + 1]),
-                         __uint_as_float(q0[4 * u + 2]), __uint_as_float(q0[4 * u + 3]));
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int quad = half * 16 + 8 + u;
-          red_add_v4_f32(dst + quad * (kB * 4), __uint_as_float(q1[4 * u]), __uint_as_float(q1[4 * u + 1]),
-                         __uint_as_float(q1[4 * u + 2]), __uint_as_float(q1[4 * u + 3]));
-        }
+        for (int x = 0; x < 32; ++x) q0[x] = q1[x] = 0u;
       }
+      reg_fence(q0);
+      reg_fence(q1);
       tc_fence_before();
       mbar_arrive(&bars[kYFree]);
+      float* dst = p.dq_acc + ((static_cast<int64_t>(b) * p.Hq + pend_h) * p.nQB + pend_i) * (kB * kD) + r * 4;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        red_add_v4_f32(dst + (c0 / 4 + u) * (kB * 4), __uint_as_float(q0[4 * u]), __uint_as_float(q0[4 * u + 1]),
+                       __uint_as_float(q0[4 * u + 2]), __uint_as_float(q0[4 * u + 3]));
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        red_add_v4_f32(dst + (c0 / 4 + 8 + u) * (kB * 4), __uint_as_float(q1[4 * u]), __uint_as_float(q1[4 * u + 1]),
+                       __uint_as_float(q1[4 * u + 2]), __uint_as_float(q1[4 * u + 3]));
       pending = false;
     };
 
@@ -373,40 +372,41 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       const bool okq = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull + st], (n >> 1) & 1, abort_flag, p.err,
                                                          wait_tag(0, kQFull + st, n)));
       const uint32_t qi = misc[8 + st];
-      if (bar_or(1, 128, !okq || *abort_flag != 0) || qi == kEndMarker) break;
+      if (bar_or(1, 256, !okq || *abort_flag != 0) || qi == kEndMarker) break;
       const int i = static_cast<int>(qi);
       const int h = static_cast<int>(misc[6 + st]);
-      const float* sZl2 = sStats + st * 384;
-      const float* sThr = sZl2 + 128;
-      const float* sDv = sZl2 + 256;
-      // test pass over S^T (one batched TMEM load of the row). Legal entries:
-      // query column c >= key row t on the diagonal tile; padded query rows
-      // carry an infinite threshold and never count
+      const float4* zl2_4 = reinterpret_cast<const float4*>(sStats + st * 384 + c0);
+      const float4* thr_4 = reinterpret_cast<const float4*>(sStats + st * 384 + 128 + c0);
+      const float4* dv_4 = reinterpret_cast<const float4*>(sStats + st * 384 + 256 + c0);
+      // test over this half of the S^T row. Legal entries: query column
+      // c >= key row r on the diagonal tile; padded query rows carry an
+      // infinite threshold and never count
       const bool oks = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], n & 1, abort_flag, p.err, wait_tag(0, kSFull, n)));
-      const int lim = (i == j) ? t : 0;
-      bool vote = false;
-      uint32_t sr[4][32];
+      const int lim = ((i == j) ? r : 0) - c0;  // first legal column of this half
+      uint32_t sr[2][32];
       if (oks) {
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tX + lane_addr + c * 32, sr[c]);
+        tmem_ld32(tX + lane_addr + c0, sr[0]);
+        tmem_ld32(tX + lane_addr + c0 + 32, sr[1]);
         tmem_ld_wait(sr[0]);
       } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int x = 0; x < 32; ++x) sr[c][x] = 0u;
+        for (int x = 0; x < 32; ++x) sr[0][x] = sr[1][x] = 0u;
       }
+      reg_fence(sr[0]);
+      reg_fence(sr[1]);
+      bool vote = false;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+      for (int x4 = 0; x4 < 16; ++x4) {
+        const float4 tv = thr_4[x4];
+        const float th[4] = {tv.x, tv.y, tv.z, tv.w};
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int col = c * 32 + x;
-          vote |= (col >= lim) && (__uint_as_float(sr[c][x]) >= sThr[col]);
+        for (int e = 0; e < 4; ++e) {
+          const int x = 4 * x4 + e;
+          vote |= (x >= lim) && (__uint_as_float(sr[x >> 5][x & 31]) >= th[e]);
         }
-      const bool keep = bar_or(1, 128, vote);
+      }
+      const bool keep = bar_or(1, 256, vote);
       if (tid == 0) {
         misc[4] = (static_cast<uint32_t>(n) << 16) | (static_cast<uint32_t>(kc) & 0xffff);
         if (mbar_wait(&bars[kDecEmpty], (n & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty, n))) {
@@ -433,64 +433,65 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       }
 
       // P^T = exp2(S^T log2e - z log2e) on legal entries, as bf16 pairs: kept
-      // in registers for dS and written over S^T in X for the dV MMA (chunk c
-      // of P^T, 16 columns, lands on S^T columns already read)
-      uint32_t pp[64];
+      // in registers for dS and written over S^T in X for the dV MMA. Both
+      // halves finished reading S^T before the vote, so the packed P^T
+      // columns [32 half, 32 half + 32) may overwrite either half's S^T.
+      uint32_t pp[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int x4 = 0; x4 < 16; ++x4) {
+        const float4 zv = zl2_4[x4];
+        const float zz[4] = {zv.x, zv.y, zv.z, zv.w};
+        float pv[4];
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          const int col = c * 32 + x;
-          const float p0 = (col >= lim) ? ex2_approx(fmaf(__uint_as_float(sr[c][x]), kLog2e, -sZl2[col])) : 0.0f;
-          const float p1 = (col + 1 >= lim) ? ex2_approx(fmaf(__uint_as_float(sr[c][x + 1]), kLog2e, -sZl2[col + 1])) : 0.0f;
-          pp[c * 16 + (x >> 1)] = pack_bf16x2(p0, p1);
+        for (int e = 0; e < 4; ++e) {
+          const int x = 4 * x4 + e;
+          pv[e] = (x >= lim) ? ex2_approx(fmaf(__uint_as_float(sr[x >> 5][x & 31]), kLog2e, -zz[e])) : 0.0f;
         }
-        tmem_st16(tX + lane_addr + c * 16, &pp[c * 16]);
+        pp[2 * x4] = pack_bf16x2(pv[0], pv[1]);
+        pp[2 * x4 + 1] = pack_bf16x2(pv[2], pv[3]);
       }
+      tmem_st16(tX + lane_addr + half * 32, &pp[0]);
+      tmem_st16(tX + lane_addr + half * 32 + 16, &pp[16]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars[kPtFull]);
 
       if (pending) drain();
 
-      // dS^T = P^T (dP^T - D) -> bf16 into the dS^T tile
+      // dS^T = P^T (dP^T - D) -> bf16 into this half's chunk of the dS^T tile
       const bool okd = __all_sync(0xffffffffu, mbar_wait(&bars[kDpFull], kc & 1, abort_flag, p.err, wait_tag(0, kDpFull, kc)));
-      tc_fence_after();
+      uint32_t dp[2][32];
+      if (okd) {
+        tc_fence_after();
+        tmem_ld32(tY + lane_addr + c0, dp[0]);
+        tmem_ld32(tY + lane_addr + c0 + 32, dp[1]);
+        tmem_ld_wait(dp[0]);
+      } else {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t dp[2][32];
-        if (okd) {
-          tmem_ld32(tY + lane_addr + half * 64, dp[0]);
-          tmem_ld32(tY + lane_addr + half * 64 + 32, dp[1]);
-          tmem_ld_wait(dp[0]);
-        } else {
+        for (int x = 0; x < 32; ++x) dp[0][x] = dp[1][x] = 0u;
+      }
+      reg_fence(dp[0]);
+      reg_fence(dp[1]);
+      const uint32_t rowb = aDS + half * kChunk + r * 128;
 #pragma unroll
-          for (int x = 0; x < 32; ++x) dp[0][x] = dp[1][x] = 0u;
-        }
-        reg_fence(dp[0]);
-        reg_fence(dp[1]);
+      for (int u = 0; u < 8; ++u) {            // 16-byte unit u: queries c0 + 8u .. + 8
+        uint32_t pk[4];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = half * 2 + cc;
-          uint32_t pk[16];
+        for (int e2 = 0; e2 < 2; ++e2) {
+          const float4 dv = dv_4[2 * u + e2];
+          const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
-          for (int x = 0; x < 32; x += 2) {
-            const int col = c * 32 + x;
-            const uint32_t w = pp[c * 16 + (x >> 1)];
+          for (int e = 0; e < 4; e += 2) {
+            const int x = 8 * u + 4 * e2 + e;
+            const uint32_t w = pp[x >> 1];
             const float p0 = __uint_as_float(w << 16);
             const float p1 = __uint_as_float(w & 0xFFFF0000u);
-            const float d0 = p0 * (__uint_as_float(dp[cc][x]) - sDv[col]);
-            const float d1 = p1 * (__uint_as_float(dp[cc][x + 1]) - sDv[col + 1]);
-            pk[x >> 1] = pack_bf16x2(d0, d1);
-          }
-          // queries [32c, 32c+32): chunk c / 2, 16-byte units (c & 1) * 4 + 0..3
-          const uint32_t rowb = aDS + (c >> 1) * kChunk + t * 128;
-#pragma unroll
-          for (int u4 = 0; u4 < 4; ++u4) {
-            const uint32_t u = (c & 1) * 4 + u4;
-            st_shared_v4(rowb + ((u ^ (t & 7)) << 4), pk[4 * u4], pk[4 * u4 + 1], pk[4 * u4 + 2], pk[4 * u4 + 3]);
+            const float d0 = p0 * (__uint_as_float(dp[x >> 5][x & 31]) - dd[e]);
+            const float d1 = p1 * (__uint_as_float(dp[(x + 1) >> 5][(x + 1) & 31]) - dd[e + 1]);
+            pk[2 * e2 + (e >> 1)] = pack_bf16x2(d0, d1);
           }
         }
+        st_shared_v4(rowb + ((u ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -504,9 +505,9 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
     }
     if (pending && !*abort_flag) drain();
 
-    // dK_j, dV_j (key row t) -> bf16
+    // dK_j, dV_j (key row r, this half's 64 columns) -> bf16
     const bool okdone = __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0, abort_flag, p.err, wait_tag(0, kDone, 0)));
-    const int krow = j * kB + t;
+    const int krow = j * kB + r;
     if (okdone && !*abort_flag) {
       tc_fence_after();
       const bool any_kept = kc > 0;            // dK/dV TMEM untouched when nothing was retained
@@ -517,17 +518,17 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         const uint32_t base = which == 0 ? tDK : tDV;
         __nv_bfloat16* outr = which == 0 ? dkr : dvr;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(base + lane_addr + c * 32, r);
-          tmem_ld_wait(r);
-          reg_fence(r);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(base + lane_addr + c0 + c * 32, rr);
+          tmem_ld_wait(rr);
+          reg_fence(rr);
           if (krow < p.N) {
             uint32_t pk[16];
 #pragma unroll
             for (int x = 0; x < 32; x += 2)
-              pk[x >> 1] = any_kept ? pack_bf16x2(__uint_as_float(r[x]), __uint_as_float(r[x + 1])) : 0u;
-            uint4* d4 = reinterpret_cast<uint4*>(outr + c * 32);
+              pk[x >> 1] = any_kept ? pack_bf16x2(__uint_as_float(rr[x]), __uint_as_float(rr[x + 1])) : 0u;
+            uint4* d4 = reinterpret_cast<uint4*>(outr + c0 + c * 32);
 #pragma unroll
             for (int u = 0; u < 4; ++u) d4[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
           }
