@@ -5,16 +5,20 @@
 // A.1, "Fused forward execution"); every legal tile is scored, and only a
 // retained tile loads V and runs the online-softmax update and PV.
 //
-// Warp roles (192 threads):
-//   warps 0-3  "softmax": thread t owns query row t (= TMEM lane t). Reads
-//              S from TMEM, applies the causal mask, computes the row max,
-//              votes on the skip test, and for retained tiles computes
-//              P = exp(S - m) into shared memory and updates m, l.
-//   warp 4     TMA producer: Q once, K tiles two ahead, V only after the
-//              vote retained the tile.
-//   warp 5     tcgen05 issuer: S_t = Q K_t^T into one of two TMEM S buffers
-//              (two tiles ahead of the vote), O += P V_t for retained tiles.
-// TMEM: S0 = cols [0,128), S1 = [128,256), O = [256, 256 + D).
+// Warp roles (320 threads):
+//   warps 0-7  softmax, two warpgroups: warps 0-3 take key columns [0, 64)
+//              of every tile, warps 4-7 columns [64, 128); (warp, lane) owns
+//              TMEM lane r = 32 (warp % 4) + lane = query row r. Per tile the
+//              groups exchange their row maxima (and the previous retained
+//              tile's row sums) through shared memory, both evaluate the same
+//              skip test, and for a retained tile each writes its half of
+//              P = exp(S - m) as packed bf16 over S in TMEM.
+//   warp 8     TMA producer, polling: Q once, K as far ahead as the ring
+//              allows (independent of the votes), V only for retained tiles.
+//   warp 9     tcgen05 issuer: S_t = Q K_t^T into one of three TMEM S buffers
+//              (up to three tiles ahead of the softmax), O += P V_t for retained tiles
+//              with P read straight from TMEM.
+// TMEM: S buffers at cols [0,128), [128,256), [256,384); O = [384, 384 + D).
 //
 // Numerics: scores are accumulated in fp32 from bf16 operands. The online
 // state is kept in base 2: m2 is a reference maximum (in log2 units) and l
@@ -33,37 +37,46 @@ namespace {
 
 constexpr int kBQ = 128;
 constexpr int kBK = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kNS = 3;                          // TMEM S buffers
 constexpr uint32_t kChunkBytes = 128 * 128;     // 128 rows x 64 bf16 (one swizzle column)
-constexpr uint32_t kPBytes = kBQ * kBK * 2;     // P tile, bf16
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;       // log2 units
 
+template <int D>
+struct Cfg {
+  static constexpr int NK = D == 128 ? 3 : 4;   // K ring stages
+  static constexpr int NV = D == 128 ? 2 : 4;   // V ring stages
+};
+
 enum Bar {
   kQFull = 0,
-  kKFull = 1,     // 2
-  kKEmpty = 3,    // 2
-  kVFull = 5,     // 2
-  kVEmpty = 7,    // 2
-  kSFull = 9,     // 2
-  kSEmpty = 11,   // 2
-  kDecFull = 13,  // 2
-  kDecEmpty = 15, // 2
-  kPFull = 17,    // 2
-  kPEmpty = 19,   // 2
-  kMmaDone = 21,
-  kNumBars = 22
+  kKFull = 1,            // 4 (ring, up to 4 stages)
+  kKEmpty = 5,           // 4
+  kVFull = 9,            // 4
+  kVEmpty = 13,          // 4
+  kSFull = 17,           // 3 (per S buffer)
+  kSDone = 20,           // 3 (per S buffer, 256 arrivals): both softmax groups are done
+                         // with the buffer's tile (P written if retained, S read if skipped);
+                         // one phase per use of the buffer, so its parity cannot alias
+  kPvDone = 23,          // PV of a retained tile completed (MMA commit)
+  kDecFull = 24,         // 2
+  kDecEmpty = 26,        // 2 (producer + MMA)
+  kMmaDone = 28,
+  kNumBars = 29
 };
 
 template <int D>
 struct Layout {
   static constexpr uint32_t kTile = kBQ * D * 2;   // Q / K / V tile bytes
   static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kTile;       // 2 stages
-  static constexpr uint32_t kV = kK + 2 * kTile;   // 2 stages
-  static constexpr uint32_t kP = kV + 2 * kTile;   // 2 buffers
-  static constexpr uint32_t kBars = kP + 2 * kPBytes;
+  static constexpr uint32_t kK = kQ + kTile;
+  static constexpr uint32_t kV = kK + Cfg<D>::NK * kTile;
+  static constexpr uint32_t kX = kV + Cfg<D>::NV * kTile;          // exchange area
+  static constexpr uint32_t kXMax = kX;                             // [2 parity][2 groups][128] float
+  static constexpr uint32_t kXSum = kX + 2 * 2 * 128 * 4;           // [2 parity][2 groups][128] float
+  static constexpr uint32_t kBars = kXSum + 2 * 2 * 128 * 4;
   static constexpr uint32_t kMisc = kBars + kNumBars * 8;
   static constexpr uint32_t kEnd = kMisc + 64;
   static constexpr uint32_t kAlloc = kEnd + 1024;  // slack for 1024-byte alignment
@@ -79,11 +92,13 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
 // per SM: the shared-memory footprint alone must rule out a second one.
 static_assert(Layout<64>::kAlloc > 116 * 1024 && Layout<128>::kAlloc > 116 * 1024,
               "forward CTA must exclude a second resident CTA per SM");
-static_assert(Layout<128>::kAlloc <= 232448, "forward CTA exceeds shared memory");
+static_assert(Layout<64>::kAlloc <= 232448 && Layout<128>::kAlloc <= 232448, "forward CTA exceeds shared memory");
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_constant__ FwdTcParams p) {
   using L = Layout<D>;
+  constexpr int NK = Cfg<D>::NK;
+  constexpr int NV = Cfg<D>::NV;
   constexpr int NCH = D / 64;       // 128-byte chunks per row of Q/K/V
   constexpr int KSTEPS = D / 16;    // QK^T k-steps
   extern __shared__ uint8_t smem_raw[];
@@ -92,7 +107,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
   uint8_t* sQ = smem + L::kQ;
   uint8_t* sK = smem + L::kK;
   uint8_t* sV = smem + L::kV;
-  uint8_t* sP = smem + L::kP;
+  float* xmax = reinterpret_cast<float*>(smem + L::kXMax);
+  float* xsum = reinterpret_cast<float*>(smem + L::kXSum);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L::kMisc);
   // misc[0] TMEM base, misc[1] abort flag, misc[2..4] progress markers of the
@@ -119,12 +135,11 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
   if (tid == 0) {
     for (int x = 0; x < kNumBars; ++x) {
       uint32_t cnt = 1;
-      if (x == kSEmpty || x == kSEmpty + 1 || x == kPFull || x == kPFull + 1) cnt = kBQ;
+      if (x >= kSDone && x < kSDone + kNS) cnt = 256;
       if (x == kDecEmpty || x == kDecEmpty + 1) cnt = 2;
       mbar_init(&bars[x], cnt);
     }
-    misc[1] = 0;
-    misc[2] = misc[3] = misc[4] = 0;
+    for (int x = 1; x < 16; ++x) misc[x] = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -135,10 +150,10 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
-  const uint32_t tmem_o = tmem + 256;
+  const uint32_t tmem_o = tmem + kNS * 128;
 
-  if (warp == 4) {
-    // ===================== TMA producer =====================
+  if (warp == 8) {
+    // ===================== TMA producer (polling) =====================
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
@@ -147,88 +162,117 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       for (int c = 0; c < NCH; ++c)
         tma_load_4d(sQ + c * kChunkBytes, &p.tm_q, &bars[kQFull], c * 64, h, q0, b);
       misc[2] = 0x10000u;
-      auto load_k = [&](int t) -> bool {
-        const int s = t & 1;
-        if (!mbar_wait(&bars[kKEmpty + s], ((t >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(1, kKEmpty + s, t))) return false;
-        mbar_expect_tx(&bars[kKFull + s], L::kTile);
-        for (int c = 0; c < NCH; ++c)
-          tma_load_4d(sK + s * L::kTile + c * kChunkBytes, &p.tm_k, &bars[kKFull + s], c * 64, hk,
-                      (j_diag - t) * kBK, b);
-        misc[2] = 0x20000u | t;
-        return true;
-      };
-      bool ok = load_k(0);
-      if (ok && T > 1) ok = load_k(1);
-      int kc = 0;
-      for (int t = 0; ok && t < T; ++t) {
-        const int s = t & 1;
-        if (!mbar_wait(&bars[kDecFull + s], (t >> 1) & 1, abort_flag, p.err, wait_tag(1, kDecFull + s, t))) { ok = false; break; }
-        const uint32_t keep = misc[5 + s];
-        mbar_arrive(&bars[kDecEmpty + s]);
-        misc[2] = 0x30000u | t;
-        if (keep) {
-          const int vs = kc & 1;
-          if (!mbar_wait(&bars[kVEmpty + vs], ((kc >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(1, kVEmpty + vs, kc))) { ok = false; break; }
-          mbar_expect_tx(&bars[kVFull + vs], L::kTile);
-          for (int c = 0; c < NCH; ++c)
-            tma_load_4d(sV + vs * L::kTile + c * kChunkBytes, &p.tm_v, &bars[kVFull + vs], c * 64,
-                        hk, (j_diag - t) * kBK, b);
-          ++kc;
+      int next_k = 0, next_d = 0, v_issued = 0, v_req = 0;
+      int vq[8];                         // retained tiles waiting for their V load
+      uint64_t idle_since = global_timer_ns();
+      bool ok = true;
+      while (ok && (next_k < T || next_d < T || v_issued < v_req)) {
+        bool progress = false;
+        if (next_k < T) {
+          const int s = next_k % NK;
+          if (mbar_test(&bars[kKEmpty + s], ((next_k / NK) & 1) ^ 1)) {
+            mbar_expect_tx(&bars[kKFull + s], L::kTile);
+            for (int c = 0; c < NCH; ++c)
+              tma_load_4d(sK + s * L::kTile + c * kChunkBytes, &p.tm_k, &bars[kKFull + s], c * 64, hk,
+                          (j_diag - next_k) * kBK, b);
+            ++next_k;
+            progress = true;
+          }
         }
-        if (t + 2 < T && !load_k(t + 2)) { ok = false; break; }
+        if (next_d < T && v_req - v_issued < 8) {
+          const int s = next_d & 1;
+          if (mbar_test(&bars[kDecFull + s], (next_d >> 1) & 1)) {
+            const uint32_t keep = misc[5 + s];
+            mbar_arrive(&bars[kDecEmpty + s]);
+            if (keep) vq[v_req++ & 7] = next_d;
+            ++next_d;
+            progress = true;
+          }
+        }
+        if (v_issued < v_req) {
+          const int s = v_issued % NV;
+          if (mbar_test(&bars[kVEmpty + s], ((v_issued / NV) & 1) ^ 1)) {
+            const int t = vq[v_issued & 7];
+            mbar_expect_tx(&bars[kVFull + s], L::kTile);
+            for (int c = 0; c < NCH; ++c)
+              tma_load_4d(sV + s * L::kTile + c * kChunkBytes, &p.tm_v, &bars[kVFull + s], c * 64, hk,
+                          (j_diag - t) * kBK, b);
+            ++v_issued;
+            progress = true;
+          }
+        }
+        misc[2] = (static_cast<uint32_t>(next_k) << 20) | (static_cast<uint32_t>(next_d) << 10) |
+                  static_cast<uint32_t>(v_issued & 0x3ff);
+        if (progress) {
+          idle_since = global_timer_ns();
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (global_timer_ns() - idle_since > kWaitLimitNs) {
+          *abort_flag = 1;
+          if (atomicCAS(p.err, 0, kErrTimeout) == 0) {
+            p.err[1] = wait_tag(1, 0xff, next_d);
+            p.err[2] = static_cast<int>(blockIdx.x);
+            for (int x = 0; x < 3; ++x) p.err[4 + x] = misc[2 + x];
+          }
+          ok = false;
+        }
       }
       if (!ok) drain_pause_ns(50000);   // let copies already issued land
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ===================== tcgen05 issuer =====================
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       auto issue_qk = [&](int t) -> bool {
-        const int s = t & 1;
-        if (!mbar_wait(&bars[kKFull + s], (t >> 1) & 1, abort_flag, p.err, wait_tag(2, kKFull + s, t))) return false;
-        if (!mbar_wait(&bars[kSEmpty + s], ((t >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(2, kSEmpty + s, t))) return false;
+        const int ks = t % NK;
+        if (!mbar_wait(&bars[kKFull + ks], (t / NK) & 1, abort_flag, p.err, wait_tag(2, kKFull + ks, t))) return false;
         tc_fence_after();
+        const uint32_t sb = tmem + (t % kNS) * 128;
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          const uint64_t a = sdesc_sw128(sQa + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sKa + s * L::kTile + off, 16, 1024);
-          umma_bf16_ss(tmem + s * 128, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(sb, sdesc_sw128(sQa + off, 16, 1024), sdesc_sw128(sKa + ks * L::kTile + off, 16, 1024),
+                       idesc_qk, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars[kSFull + s]);
-        umma_commit(&bars[kKEmpty + s]);
+        umma_commit(&bars[kSFull + (t % kNS)]);
+        umma_commit(&bars[kKEmpty + ks]);
         misc[3] = 0x20000u | t;
         return true;
       };
       bool ok = mbar_wait(&bars[kQFull], 0, abort_flag, p.err, wait_tag(2, kQFull, 0));
-      if (ok) misc[3] = 0x10000u;
-      if (ok) ok = issue_qk(0);
-      if (ok && T > 1) ok = issue_qk(1);
+      for (int t = 0; ok && t < kNS && t < T; ++t) ok = issue_qk(t);
       int kc = 0;
       for (int t = 0; ok && t < T; ++t) {
-        const int s = t & 1;
-        if (!mbar_wait(&bars[kDecFull + s], (t >> 1) & 1, abort_flag, p.err, wait_tag(2, kDecFull + s, t))) { ok = false; break; }
-        const uint32_t keep = misc[5 + s];
-        mbar_arrive(&bars[kDecEmpty + s]);
-        if (t + 2 < T && !issue_qk(t + 2)) { ok = false; break; }
+        const int ds = t & 1;
+        if (!mbar_wait(&bars[kDecFull + ds], (t >> 1) & 1, abort_flag, p.err, wait_tag(2, kDecFull + ds, t))) { ok = false; break; }
+        const uint32_t keep = misc[5 + ds];
+        mbar_arrive(&bars[kDecEmpty + ds]);
         if (keep) {
-          const int ps = kc & 1;
-          if (!mbar_wait(&bars[kPFull + ps], (kc >> 1) & 1, abort_flag, p.err, wait_tag(2, kPFull + ps, kc))) { ok = false; break; }
-          if (!mbar_wait(&bars[kVFull + ps], (kc >> 1) & 1, abort_flag, p.err, wait_tag(2, kVFull + ps, kc))) { ok = false; break; }
+          const int vs = kc % NV;
+          if (!mbar_wait(&bars[kSDone + t % kNS], (t / kNS) & 1, abort_flag, p.err, wait_tag(2, kSDone + t % kNS, t))) { ok = false; break; }
+          if (!mbar_wait(&bars[kVFull + vs], (kc / NV) & 1, abort_flag, p.err, wait_tag(2, kVFull + vs, kc))) { ok = false; break; }
           tc_fence_after();
+          const uint32_t pb = tmem + (t % kNS) * 128;   // P as packed bf16 pairs over S
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t a = sdesc_sw128(sPa + ps * kPBytes + (kk >> 2) * kChunkBytes + (kk & 3) * 32,
-                                           16, 1024);
-            const uint64_t bd = sdesc_sw128(sVa + ps * L::kTile + kk * 2048, kChunkBytes, 1024);
-            umma_bf16_ss(tmem_o, a, bd, idesc_pv, (kc > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&bars[kPEmpty + ps]);
-          umma_commit(&bars[kVEmpty + ps]);
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_bf16_ts(tmem_o, pb + kk * 8, sdesc_sw128(sVa + vs * L::kTile + kk * 2048, kChunkBytes, 1024),
+                         idesc_pv, (kc > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bars[kPvDone]);
+          umma_commit(&bars[kVEmpty + vs]);
           misc[3] = 0x40000u | t;
           ++kc;
+        }
+        // S buffer t % 3 takes tile t + 3 once tile t's contents are consumed:
+        // the PV read P from it, or both softmax groups read the skipped S
+        if (t + kNS < T) {
+          if (keep) {
+            if (!mbar_wait(&bars[kPvDone], (kc - 1) & 1, abort_flag, p.err, wait_tag(2, kPvDone, kc - 1))) { ok = false; break; }
+          } else {
+            if (!mbar_wait(&bars[kSDone + t % kNS], (t / kNS) & 1, abort_flag, p.err, wait_tag(2, kSDone + t % kNS, t))) { ok = false; break; }
+          }
+          if (!issue_qk(t + kNS)) { ok = false; break; }
         }
       }
       // make sure every MMA issued above has finished before TMEM is freed
@@ -236,18 +280,20 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       mbar_wait(&bars[kMmaDone], 0, abort_flag, p.err, wait_tag(2, kMmaDone, 0));
     }
   } else {
-    // ===================== softmax warpgroup =====================
-    const int r = tid;                       // row within the block = TMEM lane
+    // ===================== softmax warpgroups =====================
+    const int r = ((warp & 3) << 5) | lane;     // query row within the block = TMEM lane
+    const int g = warp >> 2;                    // column group: key columns [64g, 64g + 64)
+    const int c0 = g * 64;
     const int q = q0 + r;
     const bool valid = q < p.N;
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float thr2 = p.log2_tau - log2f(static_cast<float>(q + 1));   // log2(tau / L_q)
     float m2 = -INFINITY;                    // reference maximum, log2 units
     float l = 0.0f;                          // sum of 2^(s log2e - m2) over retained keys
     int kc = 0;
+    bool prev_kept = false;
     uint32_t mask_word = 0;
     int kept_tiles = 0;
-    const uint32_t sPa = smem_u32(sP);
     const int mask_base = ((b * p.Hq + h) * p.nQB + i) * p.mask_words;
     if (tid == 0 && p.keep_mask) {
       for (int w = j_diag / 32 + 1; w < p.mask_words; ++w) p.keep_mask[mask_base + w] = 0u;
@@ -255,55 +301,51 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
 
     for (int t = 0; t < T; ++t) {
       const int j = j_diag - t;
-      const int s = t & 1;
-      uint32_t sr[4][32];
+      const int sb = t % kNS;
+      uint32_t sr[2][32];
       // tcgen05.ld is warp-collective: load only if every lane's wait succeeded
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull + s], (t >> 1) & 1, abort_flag, p.err, wait_tag(0, kSFull + s, t)));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull + sb], (t / kNS) & 1, abort_flag, p.err,
+                                                        wait_tag(0, kSFull + sb, t)));
       if (ok) {
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tmem + lane_addr + s * 128 + c * 32, sr[c]);
-          tmem_ld_wait(sr[c]);
-        }
+        tmem_ld32(tmem + sb * 128 + lane_addr + c0, sr[0]);
+        tmem_ld32(tmem + sb * 128 + lane_addr + c0 + 32, sr[1]);
+        tmem_ld_wait(sr[0]);
       } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int x = 0; x < 32; ++x) sr[c][x] = 0u;
+        for (int x = 0; x < 32; ++x) sr[0][x] = sr[1][x] = 0u;
       }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
-      tc_fence_before();
-      mbar_arrive(&bars[kSEmpty + s]);
-      if (tid == 0) misc[4] = (ok ? 0x10000u : 0x90000u) | t;
+      reg_fence(sr[0]);
+      reg_fence(sr[1]);
 
-      // causal mask: key k = j*128 + c is legal iff k <= q
-      const int lim = q - j * kBK;           // largest legal column index
-      const bool has_key = valid && lim >= 0;
-      float rmax = -INFINITY;
+      // causal mask: key k = j*128 + c is legal iff k <= q; this group's
+      // columns are c = c0 + x
+      const int lim = q - j * kBK - c0;       // largest legal x
+      const bool has_key = valid && q >= j * kBK;
+      float pmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const float v = (c * 32 + x <= lim) ? __uint_as_float(sr[c][x]) : -INFINITY;
-          sr[c][x] = __float_as_uint(v);
-          rmax = fmaxf(rmax, v);
-        }
+      for (int x = 0; x < 64; ++x) {
+        const float v = (x <= lim) ? __uint_as_float(sr[x >> 5][x & 31]) : -INFINITY;
+        sr[x >> 5][x & 31] = __float_as_uint(v);
+        pmax = fmaxf(pmax, v);
+      }
+      const int par = t & 1;
+      xmax[(par * 2 + g) * 128 + r] = pmax;
+      // exchange barrier; the OR of the abort flag keeps both groups' exits in step
+      if (bar_or(1, 256, *abort_flag != 0)) break;
+      if (tid == 0) misc[4] = 0x10000u | t;
+      if (prev_kept) l += xsum[((par ^ 1) * 2 + 0) * 128 + r] + xsum[((par ^ 1) * 2 + 1) * 128 + r];
+      const float rmax = fmaxf(xmax[(par * 2 + 0) * 128 + r], xmax[(par * 2 + 1) * 128 + r]);
       const float rmax2 = rmax * kLog2e;
       // retain iff the row's largest contribution ratio reaches tau / L_q;
       // an empty retained set (l = 0) always retains
       const bool vote = has_key && (l == 0.0f || rmax2 - (m2 + lg2_approx(l)) >= thr2);
-      const bool keep = bar_or(1, kBQ, vote);
-      if (tid == 0) misc[4] = 0x20000u | t;
-      // every softmax thread must leave at the same tile: OR the flag through a barrier
-      if (bar_or(1, kBQ, *abort_flag != 0)) break;
+      const bool keep = bar_or(1, 256, vote);
 
       if (tid == 0) {
-        if (mbar_wait(&bars[kDecEmpty + s], ((t >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty + s, t))) {
-          misc[5 + s] = keep ? 1u : 0u;
-          mbar_arrive(&bars[kDecFull + s]);
-          misc[4] = 0x30000u | t;
+        if (mbar_wait(&bars[kDecEmpty + par], ((t >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty + par, t))) {
+          misc[5 + par] = keep ? 1u : 0u;
+          mbar_arrive(&bars[kDecFull + par]);
         }
         if (keep) {
           mask_word |= 1u << (j & 31);
@@ -314,7 +356,12 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
           mask_word = 0;
         }
       }
-      if (!keep) continue;
+      if (!keep) {
+        tc_fence_before();
+        mbar_arrive(&bars[kSDone + sb]);
+        prev_kept = false;
+        continue;
+      }
 
       // ---- online-softmax update for a retained tile
       float new_m2 = m2;
@@ -329,82 +376,76 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       }
       const float alpha = rescale ? ex2_approx(m2 - new_m2) : 1.0f;
       l *= alpha;
-      // O rows of this warp are rescaled together (TMEM access is warp-collective)
+      // O rows of this warp are rescaled together (TMEM access is warp-collective);
+      // each group rescales its half of the D columns
       if (kc > 0 && __any_sync(0xffffffffu, rescale)) {
-        {
-          // O holds PV of earlier retained tiles: wait for the last one
-          mbar_wait(&bars[kPEmpty + ((kc - 1) & 1)], ((kc - 1) >> 1) & 1, abort_flag, p.err, wait_tag(0, kPEmpty + ((kc - 1) & 1), kc));
-          tc_fence_after();
+        mbar_wait(&bars[kPvDone], (kc - 1) & 1, abort_flag, p.err, wait_tag(0, kPvDone, kc));
+        tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem_o + lane_addr + c * 32, o);
-            tmem_ld_wait(o);
-            reg_fence(o);
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t o[32];
+          const uint32_t oaddr = tmem_o + lane_addr + g * (D / 2) + c * 32;
+          tmem_ld32(oaddr, o);
+          tmem_ld_wait(o);
+          reg_fence(o);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            tmem_st32(tmem_o + lane_addr + c * 32, o);
-          }
-          tmem_st_wait();
+          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+          tmem_st32(oaddr, o);
         }
+        tmem_st_wait();
       }
       m2 = new_m2;
 
-      // P buffer kc & 1 is free once PV(kc - 2) has completed
-      mbar_wait(&bars[kPEmpty + (kc & 1)], ((kc >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(0, kPEmpty + (kc & 1), kc));
+      // P = 2^(s log2e - m2) as packed bf16 pairs over this tile's S buffer:
+      // key column c goes to packed column c / 2, so this group writes packed
+      // columns [32g, 32g + 32); both groups finished reading S before the vote
       const float neg_m2 = has_key ? -m2 : 0.0f;
-      float psum = 0.0f;
-      const uint32_t prow = sPa + (kc & 1) * kPBytes + r * 128;
+      float ps = 0.0f;
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          float a = has_key ? ex2_approx(fmaf(__uint_as_float(sr[c][x]), kLog2e, neg_m2)) : 0.0f;
-          float bb = has_key ? ex2_approx(fmaf(__uint_as_float(sr[c][x + 1]), kLog2e, neg_m2)) : 0.0f;
-          psum += a + bb;
-          pk[x >> 1] = pack_bf16x2(a, bb);
-        }
-        // keys [32c, 32c + 32): chunk c / 2, 16-byte units u = (c & 1) * 4 + 0..3
-        const uint32_t chunk = prow + (c >> 1) * kChunkBytes;
-#pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
-          const uint32_t u = (c & 1) * 4 + u4;
-          st_shared_v4(chunk + ((u ^ (r & 7)) << 4), pk[u4 * 4 + 0], pk[u4 * 4 + 1], pk[u4 * 4 + 2],
-                       pk[u4 * 4 + 3]);
-        }
+      for (int x = 0; x < 64; x += 2) {
+        const float a = has_key ? ex2_approx(fmaf(__uint_as_float(sr[x >> 5][x & 31]), kLog2e, neg_m2)) : 0.0f;
+        const float bb = has_key ? ex2_approx(fmaf(__uint_as_float(sr[x >> 5][(x + 1) & 31]), kLog2e, neg_m2)) : 0.0f;
+        ps += a + bb;
+        pk[x >> 1] = pack_bf16x2(a, bb);
       }
-      l += psum;
-      fence_proxy_async_smem();
+      tmem_st16(tmem + sb * 128 + lane_addr + g * 32, &pk[0]);
+      tmem_st16(tmem + sb * 128 + lane_addr + g * 32 + 16, &pk[16]);
+      xsum[(par * 2 + g) * 128 + r] = ps;
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars[kPFull + (kc & 1)]);
+      mbar_arrive(&bars[kSDone + sb]);
+      prev_kept = true;
       ++kc;
     }
 
     // ---- epilogue: O = acc / l (bf16), z = (m2 + log2 l) ln 2, mask, stats
-    if (!*abort_flag) {
-      if (kc > 0) mbar_wait(&bars[kPEmpty + ((kc - 1) & 1)], ((kc - 1) >> 1) & 1, abort_flag, p.err, wait_tag(0, kPEmpty + ((kc - 1) & 1), kc));
+    const bool aborted = bar_or(1, 256, *abort_flag != 0);   // also publishes the last sums
+    if (!aborted) {
+      if (prev_kept) l += xsum[(((T - 1) & 1) * 2 + 0) * 128 + r] + xsum[(((T - 1) & 1) * 2 + 1) * 128 + r];
+      if (kc > 0) mbar_wait(&bars[kPvDone], (kc - 1) & 1, abort_flag, p.err, wait_tag(0, kPvDone, kc));
       tc_fence_after();
       const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + b * p.o_sb +
                             static_cast<int64_t>(q) * p.o_sn + h * p.o_sh;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem_o + lane_addr + c * 32, o);
+        const int col = g * (D / 2) + c * 32;
+        tmem_ld32(tmem_o + lane_addr + col, o);
         tmem_ld_wait(o);
         reg_fence(o);
         if (valid) {
-          uint32_t pk[16];
+          uint32_t pko[16];
 #pragma unroll
           for (int x = 0; x < 32; x += 2)
-            pk[x >> 1] = pack_bf16x2(__uint_as_float(o[x]) * inv_l, __uint_as_float(o[x + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+            pko[x >> 1] = pack_bf16x2(__uint_as_float(o[x]) * inv_l, __uint_as_float(o[x + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          for (int u = 0; u < 4; ++u) dst[u] = make_uint4(pko[4 * u], pko[4 * u + 1], pko[4 * u + 2], pko[4 * u + 3]);
         }
       }
-      if (valid) p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.N + q] = (m2 + log2f(l)) * kLn2;
+      if (valid && g == 0) p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.N + q] = (m2 + log2f(l)) * kLn2;
       if (tid == 0 && p.stats) {
         const int nvalid = last_row - q0 + 1;
         atomicAdd(reinterpret_cast<unsigned long long*>(&p.stats[0]), static_cast<unsigned long long>(T));
