@@ -60,11 +60,13 @@ enum Bar {
   kSDone = 20,           // 3 (per S buffer, 256 arrivals): both softmax groups are done
                          // with the buffer's tile (P written if retained, S read if skipped);
                          // one phase per use of the buffer, so its parity cannot alias
-  kPvDone = 23,          // PV of a retained tile completed (MMA commit)
-  kDecFull = 24,         // 2
-  kDecEmpty = 26,        // 2 (producer + MMA)
-  kMmaDone = 28,
-  kNumBars = 29
+  kTileDone = 23,        // 3 (per S buffer, MMA commit once per tile after its PV, or
+                         // right away for a skipped tile): every MMA issued up to
+                         // that tile has completed; one phase per use of the buffer
+  kDecFull = 26,         // 2
+  kDecEmpty = 28,        // 2 (producer + MMA)
+  kMmaDone = 30,
+  kNumBars = 31
 };
 
 template <int D>
@@ -259,19 +261,18 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
           for (int kk = 0; kk < kBK / 16; ++kk)
             umma_bf16_ts(tmem_o, pb + kk * 8, sdesc_sw128(sVa + vs * L::kTile + kk * 2048, kChunkBytes, 1024),
                          idesc_pv, (kc > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&bars[kPvDone]);
           umma_commit(&bars[kVEmpty + vs]);
           misc[3] = 0x40000u | t;
           ++kc;
         }
+        umma_commit(&bars[kTileDone + t % kNS]);
         // S buffer t % 3 takes tile t + 3 once tile t's contents are consumed:
-        // the PV read P from it, or both softmax groups read the skipped S
+        // both softmax groups are done with it and every MMA reading it (the
+        // PV of a retained tile) has completed
         if (t + kNS < T) {
-          if (keep) {
-            if (!mbar_wait(&bars[kPvDone], (kc - 1) & 1, abort_flag, p.err, wait_tag(2, kPvDone, kc - 1))) { ok = false; break; }
-          } else {
-            if (!mbar_wait(&bars[kSDone + t % kNS], (t / kNS) & 1, abort_flag, p.err, wait_tag(2, kSDone + t % kNS, t))) { ok = false; break; }
-          }
+          if (!keep &&
+              !mbar_wait(&bars[kSDone + t % kNS], (t / kNS) & 1, abort_flag, p.err, wait_tag(2, kSDone + t % kNS, t))) { ok = false; break; }
+          if (!mbar_wait(&bars[kTileDone + t % kNS], (t / kNS) & 1, abort_flag, p.err, wait_tag(2, kTileDone + t % kNS, t))) { ok = false; break; }
           if (!issue_qk(t + kNS)) { ok = false; break; }
         }
       }
@@ -319,16 +320,23 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       reg_fence(sr[1]);
 
       // causal mask: key k = j*128 + c is legal iff k <= q; this group's
-      // columns are c = c0 + x
-      const int lim = q - j * kBK - c0;       // largest legal x
+      // columns are c = c0 + x. Only the diagonal tile (t = 0) has illegal
+      // keys: every earlier key block lies below the block's first row.
       const bool has_key = valid && q >= j * kBK;
-      float pmax = -INFINITY;
+      if (t == 0) {
+        const int lim = q - j * kBK - c0;     // largest legal x
 #pragma unroll
-      for (int x = 0; x < 64; ++x) {
-        const float v = (x <= lim) ? __uint_as_float(sr[x >> 5][x & 31]) : -INFINITY;
-        sr[x >> 5][x & 31] = __float_as_uint(v);
-        pmax = fmaxf(pmax, v);
+        for (int x = 0; x < 64; ++x)
+          if (x > lim) sr[x >> 5][x & 31] = __float_as_uint(-INFINITY);
       }
+      // row maximum of this half: eight independent chains, then a tree
+      float mx[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(sr[0][e]);
+#pragma unroll
+      for (int x = 8; x < 64; ++x) mx[x & 7] = fmaxf(mx[x & 7], __uint_as_float(sr[x >> 5][x & 31]));
+      const float pmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const int par = t & 1;
       xmax[(par * 2 + g) * 128 + r] = pmax;
       // exchange barrier; the OR of the abort flag keeps both groups' exits in step
@@ -379,7 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       // O rows of this warp are rescaled together (TMEM access is warp-collective);
       // each group rescales its half of the D columns
       if (kc > 0 && __any_sync(0xffffffffu, rescale)) {
-        mbar_wait(&bars[kPvDone], (kc - 1) & 1, abort_flag, p.err, wait_tag(0, kPvDone, kc));
+        // O holds the PVs of earlier retained tiles: wait until every MMA up
+        // to the previous tile has completed (t >= 1 since kc > 0)
+        const int tp = t - 1;
+        mbar_wait(&bars[kTileDone + tp % kNS], (tp / kNS) & 1, abort_flag, p.err, wait_tag(0, kTileDone + tp % kNS, tp));
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
@@ -399,16 +410,18 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       // P = 2^(s log2e - m2) as packed bf16 pairs over this tile's S buffer:
       // key column c goes to packed column c / 2, so this group writes packed
       // columns [32g, 32g + 32); both groups finished reading S before the vote
-      const float neg_m2 = has_key ? -m2 : 0.0f;
-      float ps = 0.0f;
+      // rows without a legal key (padding) get P = 0 through m2 = +inf
+      const float neg_m2 = has_key ? -m2 : -INFINITY;
+      float psum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       uint32_t pk[32];
 #pragma unroll
       for (int x = 0; x < 64; x += 2) {
-        const float a = has_key ? ex2_approx(fmaf(__uint_as_float(sr[x >> 5][x & 31]), kLog2e, neg_m2)) : 0.0f;
-        const float bb = has_key ? ex2_approx(fmaf(__uint_as_float(sr[x >> 5][(x + 1) & 31]), kLog2e, neg_m2)) : 0.0f;
-        ps += a + bb;
+        const float a = ex2_approx(fmaf(__uint_as_float(sr[x >> 5][x & 31]), kLog2e, neg_m2));
+        const float bb = ex2_approx(fmaf(__uint_as_float(sr[x >> 5][(x + 1) & 31]), kLog2e, neg_m2));
+        psum[(x >> 1) & 3] += a + bb;
         pk[x >> 1] = pack_bf16x2(a, bb);
       }
+      const float ps = (psum[0] + psum[1]) + (psum[2] + psum[3]);
       tmem_st16(tmem + sb * 128 + lane_addr + g * 32, &pk[0]);
       tmem_st16(tmem + sb * 128 + lane_addr + g * 32 + 16, &pk[16]);
       xsum[(par * 2 + g) * 128 + r] = ps;
@@ -423,7 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
     const bool aborted = bar_or(1, 256, *abort_flag != 0);   // also publishes the last sums
     if (!aborted) {
       if (prev_kept) l += xsum[(((T - 1) & 1) * 2 + 0) * 128 + r] + xsum[(((T - 1) & 1) * 2 + 1) * 128 + r];
-      if (kc > 0) mbar_wait(&bars[kPvDone], (kc - 1) & 1, abort_flag, p.err, wait_tag(0, kPvDone, kc));
+      if (kc > 0)
+        mbar_wait(&bars[kTileDone + (T - 1) % kNS], ((T - 1) / kNS) & 1, abort_flag, p.err,
+                  wait_tag(0, kTileDone + (T - 1) % kNS, T - 1));
       tc_fence_after();
       const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + b * p.o_sb +
