@@ -110,6 +110,35 @@ def _dist_init():
     return world, rank, local
 
 
+# DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
+# on the kernel versions in this tree. Backward: one full-size launch of this
+# workload. Decode: one launch at N_k = 8192, scaled to N_k = 131072 by the
+# key/value bytes (read once, so traffic grows with N_k; the split partials
+# are the same at both sizes). Set an entry to None when its kernel changes.
+NCU_TRAFFIC = {
+    "mala_bwd_tc_kernel": 8.36e9 + 4.16e9,
+    "mala_decode_split_kernel@131072": (2.148422e9 - 2.147484e9) + 2.147484e9 * 16 + 7.1e6,
+}
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Largest value of ``x`` over all ranks (the slowest rank's time); the
+    value itself when no process group is running."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, seconds: float) -> float:
+    """Units all ranks processed per second of the slowest rank (weak scaling:
+    every rank processes its own units_per_rank)."""
+    return units_per_rank * world / seconds
+
+
 def tile_flops(d: int = 128) -> float:
     """FLOPs of one 128 x 128 x d tile matmul (2 per multiply-add)."""
     return 2.0 * TILE * TILE * d
@@ -188,13 +217,9 @@ def run_mala(args):
     mala.check_device_error()
     fwd_times = [a.elapsed_time(b_) / 1e3 for a, b_ in evf]
     bwd_times = [a.elapsed_time(b_) / 1e3 for a, b_ in evb]
-    if world > 1:
-        tt = torch.tensor([elapsed], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed = float(tt.item())
+    elapsed = max_over_ranks(elapsed, dev)
     ms_per_step = elapsed / args.steps * 1e3
-    tokens = B * N * world * args.steps
-    value = tokens / elapsed
+    value = whole_job_rate(B * N * args.steps, world, elapsed)
 
     if args.no_extras:
         if rank == 0:
@@ -217,7 +242,8 @@ def run_mala(args):
         step(0.0)
     e1.record(stream)
     torch.cuda.synchronize()
-    dense_s = e0.elapsed_time(e1) / 1e3 / n_dense
+    dense_s = max_over_ranks(e0.elapsed_time(e1) / 1e3 / n_dense, dev)
+    dense = {"o": o.clone(), "lse": lse.clone(), "dq": dq.clone(), "dk": dk.clone(), "dv": dv.clone()}
     dense_flops = tile_flops(d) * (d_tested + d_kept + db_visit + 4 * db_kept)
 
     # end to end through the public API with pinned host buffers: inputs in,
@@ -236,7 +262,19 @@ def run_mala(args):
             outs_h[n_].copy_(x, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_s = e0.elapsed_time(e1) / 1e3
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
+
+    # fidelity against the dense (tau = 0) run on the same inputs: the
+    # retained share of each row's softmax mass is exp(z_mala - z_dense), so
+    # the omitted mass is 1 minus it; relative L2 errors of O and gradients
+    step(TAU)
+    torch.cuda.synchronize()
+    omitted = (1.0 - torch.exp(lse.double() - dense["lse"].double())).clamp_min(0.0)
+    rel = lambda a_, b_: float((a_.double() - b_.double()).norm() / b_.double().norm())
+    fidelity = {"omitted_mass_mean": float(omitted.mean()), "omitted_mass_max": float(omitted.max()),
+                "o_rel_l2": rel(o, dense["o"]), "dq_rel_l2": rel(dq, dense["dq"]),
+                "dk_rel_l2": rel(dk, dense["dk"]), "dv_rel_l2": rel(dv, dense["dv"])}
+    del dense
 
     peaks = _peaks()
     dec = None if args.no_decode else bench_decode(args, dev, stream, peaks)
@@ -270,13 +308,16 @@ def run_mala(args):
         "bwd": {"ms": kern_b * 1e3, "tflops_executed": ach_b, "frac_of_peak": ach_b / peak,
                 "tiles_visited": b_visit, "tiles_kept": b_kept, "kept_fraction": b_kept / max(b_visit, 1),
                 "slots_per_query": b_slots / (B * Hq * N)},
-        "tau0": {"ms_per_step": dense_s * 1e3, "tokens_per_s": B * N * world / dense_s,
+        "tau0": {"ms_per_step": dense_s * 1e3, "tokens_per_s": whole_job_rate(B * N, world, dense_s),
                  "tflops_executed": dense_flops / dense_s / 1e12},
+        "fidelity_vs_tau0": fidelity,
         "roofline": {"bound": "tensor", "kernel": dom[0], "achieved": dom[1],
                      "peak": peak, "unit": "TFLOP/s", "frac": dom[1] / peak,
                      "peak_source": f"{peaks['source']} bf16_tflops_sustained",
-                     "traffic": None},
-        "e2e": {"value": B * N * args.steps / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                     "traffic": (NCU_TRAFFIC.get("mala_bwd_tc_kernel")
+                                 if kern_b >= kern_f and N == 32768 else None),
+                     "traffic_note": "ncu DRAM bytes of the mala_bwd_tc_kernel launch (bytes per launch)"},
+        "e2e": {"value": whole_job_rate(B * N * args.steps, world, e2e_s), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
@@ -344,7 +385,9 @@ def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072):
             "bytes_read_per_call": kbytes + vbytes + w.batch * w.heads_q * d * 2,
             "roofline": {"bound": "hbm", "kernel": "mala_decode_split_kernel", "achieved": gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-                         "peak_source": f"{peaks['source']} hbm_gbs", "traffic": None}}
+                         "peak_source": f"{peaks['source']} hbm_gbs",
+                         "traffic": NCU_TRAFFIC.get(f"mala_decode_split_kernel@{w.seqlen_k}"),
+                         "traffic_note": "ncu DRAM bytes per launch, N_k = 8192 capture scaled by N_k"}}
 
 
 _ORACLE_INPUTS = {}
