@@ -14,7 +14,7 @@
 // Roles (320 threads): warps 0-7 compute in two warpgroups that split the
 // 128 query columns of a tile (lane t of TMEM is key row t for S^T, P^T,
 // dP^T, dS^T and query row t for the dQ part), warp 8 TMA producer
-// (polling: Q of the next tiles and dO of retained tiles), warp 9 tcgen05
+// (in order, blocking waits: Q of the next tiles and dO of retained tiles), warp 9 tcgen05
 // issuer.
 // TMEM: X = cols [0,128): S^T(n), then P^T(n) as packed bf16 in [0,64),
 // read by the dV MMA straight from TMEM; Y = [128,256): dP^T(n), then the
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
   const uint32_t tX = tmem, tY = tmem + 128, tDK = tmem + 256, tDV = tmem + 384;
 
   if (warp == 8) {
-    // ===================== producer (polling) =====================
+    // ===================== producer (in order) =====================
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
@@ -147,83 +147,63 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         }
         return false;
       };
-      int n_load = 0, n_dec = 0, kc_load = 0, n_total = -1;   // n_total known once the end marker is loaded
-      int pend_h[2], pend_i[2], pend_n = 0;                    // retained tiles waiting for their dO load
-      // (head, query block) of tile n at [n % 4]: decisions trail the Q loads
-      // by at most three tiles (a tile's Q stage is refilled only after its
-      // decision was published, and the next decision waits for this one to
-      // be read)
+      // (head, query block) of tile n at [n & 3]: Q of tile n + 2 is loaded
+      // only after the decision on tile n was read
       int info_h[4] = {0, 0, 0, 0}, info_i[4] = {0, 0, 0, 0};
-      uint64_t idle_since = global_timer_ns();
+      // Q of tile n and its row statistics into stage n & 1; the end marker
+      // instead when there is no tile n
+      auto load_q = [&](int n) -> bool {
+        const int st = n & 1;
+        int h = 0, i = 0;
+        if (!next_tile(h, i)) {
+          misc[8 + st] = kEndMarker;
+          mbar_arrive(&bars[kQFull + st]);
+          return false;
+        }
+        info_h[n & 3] = h;
+        info_i[n & 3] = i;
+        misc[6 + st] = static_cast<uint32_t>(h);
+        misc[8 + st] = static_cast<uint32_t>(i);
+        mbar_expect_tx(&bars[kQFull + st], kTile + 3 * 512);
+        for (int c = 0; c < 2; ++c)
+          tma_load_4d(sQ + st * kTile + c * kChunk, &p.tm_q, &bars[kQFull + st], c * 64, h, i * kB, b);
+        const int64_t row0 = (static_cast<int64_t>(b) * p.Hq + h) * p.Npad + static_cast<int64_t>(i) * kB;
+        float* sst = sStats + st * 384;
+        bulk_load(sst, p.zl2 + row0, 512, &bars[kQFull + st]);
+        bulk_load(sst + 128, p.t2 + row0, 512, &bars[kQFull + st]);
+        bulk_load(sst + 256, p.Dv + row0, 512, &bars[kQFull + st]);
+        return true;
+      };
+      // In order, with blocking waits: per tile n, read its decision (and
+      // load its dO when retained), then refill its Q stage with tile n + 2
+      // once tile n released it. Every wait is for the next event this role
+      // needs, so the thread sleeps in the barrier wait instead of polling.
+      int n_total = -1;                         // number of tiles, once known
+      for (int n = 0; n < 2 && n_total < 0; ++n)
+        if (!load_q(n)) n_total = n;
+      int kc_load = 0;
       bool ok = true;
-      while (ok) {
-        bool progress = false;
-        if (n_total < 0) {
-          const int st = n_load & 1;
-          if (mbar_test(&bars[kQEmpty + st], ((n_load >> 1) & 1) ^ 1)) {
-            int h = 0, i = 0;
-            if (next_tile(h, i)) {
-              info_h[n_load & 3] = h;
-              info_i[n_load & 3] = i;
-              misc[6 + st] = static_cast<uint32_t>(h);
-              misc[8 + st] = static_cast<uint32_t>(i);
-              mbar_expect_tx(&bars[kQFull + st], kTile + 3 * 512);
-              for (int c = 0; c < 2; ++c)
-                tma_load_4d(sQ + st * kTile + c * kChunk, &p.tm_q, &bars[kQFull + st], c * 64, h, i * kB, b);
-              const int64_t row0 = (static_cast<int64_t>(b) * p.Hq + h) * p.Npad + static_cast<int64_t>(i) * kB;
-              float* sst = sStats + st * 384;
-              bulk_load(sst, p.zl2 + row0, 512, &bars[kQFull + st]);
-              bulk_load(sst + 128, p.t2 + row0, 512, &bars[kQFull + st]);
-              bulk_load(sst + 256, p.Dv + row0, 512, &bars[kQFull + st]);
-            } else {
-              misc[8 + st] = kEndMarker;
-              mbar_arrive(&bars[kQFull + st]);
-              n_total = n_load;
-            }
-            ++n_load;
-            progress = true;
-          }
-        }
-        if (n_dec < n_load && (n_total < 0 || n_dec < n_total) && pend_n < 2) {
-          if (mbar_test(&bars[kDecFull], n_dec & 1)) {
-            const uint32_t keep = misc[5];
-            mbar_arrive(&bars[kDecEmpty]);
-            if (keep) {
-              pend_h[pend_n] = info_h[n_dec & 3];
-              pend_i[pend_n] = info_i[n_dec & 3];
-              ++pend_n;
-            }
-            ++n_dec;
-            progress = true;
-          }
-        }
-        if (pend_n > 0 && mbar_test(&bars[kDoEmpty], (kc_load & 1) ^ 1)) {
+      for (int n = 0; n_total < 0 || n < n_total; ++n) {
+        ok = mbar_wait(&bars[kDecFull], n & 1, abort_flag, p.err, wait_tag(1, kDecFull, n));
+        if (!ok) break;
+        const uint32_t keep = misc[5];
+        mbar_arrive(&bars[kDecEmpty]);
+        if (keep) {
+          ok = mbar_wait(&bars[kDoEmpty], (kc_load & 1) ^ 1, abort_flag, p.err, wait_tag(1, kDoEmpty, kc_load));
+          if (!ok) break;
           mbar_expect_tx(&bars[kDoFull], kTile);
           for (int c = 0; c < 2; ++c)
-            tma_load_4d(sDO + c * kChunk, &p.tm_do, &bars[kDoFull], c * 64, pend_h[0], pend_i[0] * kB, b);
-          pend_h[0] = pend_h[1];
-          pend_i[0] = pend_i[1];
-          --pend_n;
+            tma_load_4d(sDO + c * kChunk, &p.tm_do, &bars[kDoFull], c * 64, info_h[n & 3], info_i[n & 3] * kB, b);
           ++kc_load;
-          progress = true;
         }
-        misc[2] = (static_cast<uint32_t>(n_load) << 16) | (static_cast<uint32_t>(n_dec) & 0xffff);
-        if (n_total >= 0 && n_dec == n_total && pend_n == 0) break;
-        if (progress) {
-          idle_since = global_timer_ns();
-        } else if (*abort_flag) {
-          ok = false;
-        } else if (global_timer_ns() - idle_since > kWaitLimitNs) {
-          *abort_flag = 1;
-          if (atomicCAS(p.err, 0, kErrTimeout) == 0) {
-            p.err[1] = wait_tag(1, 0xff, n_dec);
-            p.err[2] = static_cast<int>(blockIdx.x);
-            for (int x = 0; x < 3; ++x) p.err[4 + x] = misc[2 + x];
-          }
-          ok = false;
+        if (n_total < 0) {
+          ok = mbar_wait(&bars[kQEmpty + (n & 1)], (n >> 1) & 1, abort_flag, p.err, wait_tag(1, kQEmpty + (n & 1), n));
+          if (!ok) break;
+          if (!load_q(n + 2)) n_total = n + 2;
         }
+        misc[2] = (static_cast<uint32_t>(n) << 16) | (static_cast<uint32_t>(kc_load) & 0xffff);
       }
-      if (!ok) drain_pause_ns(50000);
+      if (!ok) drain_pause_ns(50000);   // let copies already issued land
     }
   } else if (warp == 9) {
     // ===================== tcgen05 issuer =====================
