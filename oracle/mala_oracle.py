@@ -160,15 +160,22 @@ def causal_tiles(pos_last: int, B_k: int, n_kblocks: int) -> list:
 def forward_head(Q: np.ndarray, K: np.ndarray, V: np.ndarray, B_q: int,
                  B_k: int, tau: float, replay_mask: Optional[np.ndarray] = None,
                  blocks: Optional[Iterable[int]] = None):
-    """Algorithm 1 for one (batch, query-head) pair, causal with N_q = N_k.
+    """Algorithm 1 for one (batch, query-head) pair, causal.
 
-    Returns O [N, d], z [N], keep [nQB, nKB] bool, margin [nQB, nKB]
+    N_q <= N_k with bottom-right alignment: query q sits at position
+    q + N_k - N_q, sees keys k <= that position, and L_q = position + 1
+    (N_q = N_k is the training case L_q = q + 1; N_q = 1 is single-token
+    decoding with L_0 = N_k, "Setup"). Query blocks are formed from the
+    first query row.
+
+    Returns O [N_q, d], z [N_q], keep [nQB, nKB] bool, margin [nQB, nKB]
     (NaN where a tile is never visited). ``blocks`` restricts the query
     blocks computed (rows of other blocks are left NaN).
     """
     N_q, d = Q.shape
     N_k = K.shape[0]
-    assert N_q == N_k, "causal mode uses equal lengths"
+    assert N_q <= N_k, "causal mode needs N_q <= N_k (bottom-right alignment)"
+    off = N_k - N_q
     nQB, nKB = num_blocks(N_q, B_q), num_blocks(N_k, B_k)
     O = np.full((N_q, V.shape[1]), np.nan)
     z = np.full(N_q, np.nan)
@@ -176,8 +183,8 @@ def forward_head(Q: np.ndarray, K: np.ndarray, V: np.ndarray, B_q: int,
     margin = np.full((nQB, nKB), np.nan)
     for i in (range(nQB) if blocks is None else blocks):
         q0, q1 = i * B_q, min((i + 1) * B_q, N_q)
-        pos = np.arange(q0, q1)
-        tiles = causal_tiles(q1 - 1, B_k, nKB)
+        pos = np.arange(q0, q1) + off
+        tiles = causal_tiles(q1 - 1 + off, B_k, nKB)
         rep = None
         if replay_mask is not None:
             rep = {j: bool(replay_mask[i, j]) for j in tiles}
@@ -191,11 +198,12 @@ def forward_head(Q: np.ndarray, K: np.ndarray, V: np.ndarray, B_q: int,
 
 def forward(q, k, v, B_q: int, B_k: int, tau: float, replay_mask=None,
             heads=None):
-    """Algorithm 1 over [B, N, Hq, d] / [B, N, Hkv, d] arrays (GQA: query
-    head h reads key/value head h // (Hq / Hkv)).
+    """Algorithm 1 over [B, N_q, Hq, d] / [B, N_k, Hkv, d] arrays (GQA: query
+    head h reads key/value head h // (Hq / Hkv); N_q <= N_k, bottom-right
+    aligned as in forward_head).
 
     replay_mask: optional bool [B, Hq, nQB, nKB]. ``heads`` optionally lists
-    (b, h) pairs to compute. Returns O [B, N, Hq, d], lse [B, Hq, N],
+    (b, h) pairs to compute. Returns O [B, N_q, Hq, d], lse [B, Hq, N_q],
     keep [B, Hq, nQB, nKB], margin (same shape)."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -203,7 +211,7 @@ def forward(q, k, v, B_q: int, B_k: int, tau: float, replay_mask=None,
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
     G = Hq // Hkv
-    nQB, nKB = num_blocks(N, B_q), num_blocks(N, B_k)
+    nQB, nKB = num_blocks(N, B_q), num_blocks(k.shape[1], B_k)
     O = np.full(q.shape[:3] + (v.shape[3],), np.nan)
     lse = np.full((B, Hq, N), np.nan)
     keep = np.zeros((B, Hq, nQB, nKB), dtype=bool)
@@ -227,7 +235,8 @@ def backward_head(Q, K, V, O, dO, z, B_q: int, B_k: int, tau: float,
                   qblocks: Optional[Iterable[int]] = None):
     """Algorithm 2 for one query head against its key/value head.
 
-    Q, O, dO [N, d]; K, V [N, d]; z [N] the saved log-normaliser.
+    Q, O, dO [N_q, d]; K, V [N_k, d]; z [N_q] the saved log-normaliser;
+    N_q <= N_k, bottom-right aligned as in forward_head.
     fwd_mask  optional bool [nQB, nKB]: when given, only tiles the forward
               retained are visited (mask replay); when None every legal tile
               is visited (the page's pure form).
@@ -239,10 +248,13 @@ def backward_head(Q, K, V, O, dO, z, B_q: int, B_k: int, tau: float,
     Q, K, V, O, dO = (np.asarray(x, dtype=np.float64) for x in (Q, K, V, O, dO))
     z = np.asarray(z, dtype=np.float64)
     N, d = Q.shape
-    nQB, nKB = num_blocks(N, B_q), num_blocks(N, B_k)
+    N_k = K.shape[0]
+    assert N <= N_k, "causal mode needs N_q <= N_k (bottom-right alignment)"
+    off = N_k - N
+    nQB, nKB = num_blocks(N, B_q), num_blocks(N_k, B_k)
     D = (dO * O).sum(axis=1)                         # D_q = rowsum(dO o O)
     log_tau = _log(tau)
-    log_L = np.log(np.arange(1, N + 1, dtype=np.float64))   # L_q = q + 1
+    log_L = np.log(np.arange(1, N + 1, dtype=np.float64) + off)   # L_q = position + 1
     dQ = np.zeros_like(Q)
     dK = np.zeros_like(K)
     dV = np.zeros_like(V)
@@ -250,15 +262,15 @@ def backward_head(Q, K, V, O, dO, z, B_q: int, B_k: int, tau: float,
     margin = np.full((nQB, nKB), np.nan)
     qset = None if qblocks is None else set(qblocks)
     for j in (range(nKB) if kblocks is None else kblocks):
-        k0, k1 = j * B_k, min((j + 1) * B_k, N)
-        i_diag = k0 // B_q                           # first block with a legal row
+        k0, k1 = j * B_k, min((j + 1) * B_k, N_k)
+        i_diag = max(0, k0 - off) // B_q             # first block with a legal row
         for i in range(i_diag, nQB):                 # ascending from the diagonal
             if qset is not None and i not in qset:
                 continue
             if fwd_mask is not None and not fwd_mask[i, j]:
                 continue
             q0, q1 = i * B_q, min((i + 1) * B_q, N)
-            qpos = np.arange(q0, q1)
+            qpos = np.arange(q0, q1) + off
             kpos = np.arange(k0, k1)
             S_ji = K[k0:k1] @ Q[q0:q1].T             # recomputed key-major tile
             legal = kpos[:, None] <= qpos[None, :]
@@ -289,7 +301,7 @@ def backward(q, k, v, o, do, lse, B_q: int, B_k: int, tau: float,
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
     G = Hq // Hkv
-    nQB, nKB = num_blocks(N, B_q), num_blocks(N, B_k)
+    nQB, nKB = num_blocks(N, B_q), num_blocks(k.shape[1], B_k)
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)

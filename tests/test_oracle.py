@@ -170,20 +170,23 @@ def test_gqa_backward_sums_group():
 def _brute_forward(Q, K, V, Bq, Bk, tau):
     """The paper's test in ratio form with explicit retained key sets:
     r_qj = max_{k in J_j, legal} exp(s_qk) / sum_{k in R_q} exp(s_qk);
-    skip iff r < tau / L_q for every row with a legal key (empty R: keep)."""
-    N = Q.shape[0]
+    skip iff r < tau / L_q for every row with a legal key (empty R: keep).
+    Query row q sits at position q + N_k - N_q (bottom-right alignment), sees
+    keys k <= that position, and L_q = position + 1."""
+    N, Nk = Q.shape[0], K.shape[0]
+    off = Nk - N
     S = Q @ K.T
-    nQB, nKB = -(-N // Bq), -(-N // Bk)
+    nQB, nKB = -(-N // Bq), -(-Nk // Bk)
     keep = np.zeros((nQB, nKB), dtype=bool)
-    O = np.zeros_like(V)
+    O = np.zeros((N, V.shape[1]))
     for i in range(nQB):
         rows = list(range(i * Bq, min((i + 1) * Bq, N)))
         R = {q: [] for q in rows}
-        for j in range(min(rows[-1] // Bk, nKB - 1), -1, -1):
-            cols = list(range(j * Bk, min((j + 1) * Bk, N)))
+        for j in range(min((rows[-1] + off) // Bk, nKB - 1), -1, -1):
+            cols = list(range(j * Bk, min((j + 1) * Bk, Nk)))
             retain = False
             for q in rows:
-                legal = [k for k in cols if k <= q]
+                legal = [k for k in cols if k <= q + off]
                 if not legal:
                     continue
                 if not R[q]:
@@ -191,12 +194,12 @@ def _brute_forward(Q, K, V, Bq, Bk, tau):
                     continue
                 Z = sum(math.exp(S[q, k]) for k in R[q])
                 r = max(math.exp(S[q, k]) for k in legal) / Z
-                if not (r < tau / (q + 1)):
+                if not (r < tau / (q + off + 1)):
                     retain = True
             keep[i, j] = retain
             if retain:
                 for q in rows:
-                    R[q] += [k for k in cols if k <= q]
+                    R[q] += [k for k in cols if k <= q + off]
         for q in rows:
             w = np.array([math.exp(S[q, k]) for k in R[q]])
             O[q] = (w / w.sum()) @ V[R[q]]
@@ -411,3 +414,92 @@ def test_replay_forces_decisions_but_keeps_margins():
     flipped[3, 1] = not flipped[3, 1]
     _, _, keep3, _ = orc.forward_head(Q, K, V, 8, 8, 0.5, replay_mask=flipped)
     assert keep3[3, 1] == flipped[3, 1]
+
+
+# ------------------------------------------- bottom-right causal alignment
+# A chunk of N_q queries at the end of an N_k-key context: query q is at
+# position q + N_k - N_q ("Setup": C_q are the keys up to the query's
+# position, L_q = |C_q|; N_q = 1 is the decoding case L_0 = N_k).
+
+def _dense_bottom_right(Q, K, V):
+    q = torch.tensor(Q, dtype=torch.float64, requires_grad=True)
+    k = torch.tensor(K, dtype=torch.float64, requires_grad=True)
+    v = torch.tensor(V, dtype=torch.float64, requires_grad=True)
+    Nq, Nk = q.shape[0], k.shape[0]
+    allowed = torch.arange(Nk)[None, :] <= (torch.arange(Nq)[:, None] + (Nk - Nq))
+    s = (q @ k.T).masked_fill(~allowed, -float("inf"))
+    out = torch.softmax(s, dim=-1) @ v
+    return q, k, v, out, torch.logsumexp(s, dim=-1)
+
+
+@pytest.mark.parametrize("Nq,Nk,d,Bq,Bk", [(13, 37, 5, 4, 8), (20, 21, 4, 8, 4), (9, 40, 3, 4, 4), (1, 29, 6, 8, 8)])
+def test_bottom_right_tau_zero_is_dense(Nq, Nk, d, Bq, Bk):
+    rng = np.random.default_rng(Nq * 31 + Nk)
+    Q = rng.standard_normal((Nq, d)) * 3 / math.sqrt(d)
+    K = rng.standard_normal((Nk, d))
+    V = rng.standard_normal((Nk, d))
+    dO = rng.standard_normal((Nq, d))
+    q, k, v, out, lse = _dense_bottom_right(Q, K, V)
+    out.backward(torch.tensor(dO))
+    O, z, keep, _ = orc.forward_head(Q, K, V, Bq, Bk, 0.0)
+    assert np.abs(O - out.detach().numpy()).max() < 1e-12
+    assert np.abs(z - lse.detach().numpy()).max() < 1e-12
+    dQ, dK, dV, _, _ = orc.backward_head(Q, K, V, O, dO, z, Bq, Bk, 0.0, keep)
+    assert np.abs(dQ - q.grad.numpy()).max() < 1e-11
+    assert np.abs(dK - k.grad.numpy()).max() < 1e-11
+    assert np.abs(dV - v.grad.numpy()).max() < 1e-11
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("tau", [0.05, 0.5, 2.0])
+def test_bottom_right_matches_brute_force(seed, tau):
+    rng = np.random.default_rng(500 + seed)
+    Nk = int(rng.integers(12, 33))
+    Nq = int(rng.integers(1, Nk + 1))
+    d = int(rng.integers(2, 7))
+    Bq = int(rng.choice([1, 2, 4, 8]))
+    Bk = int(rng.choice([1, 2, 4, 8]))
+    Q = rng.standard_normal((Nq, d)) * 4 / math.sqrt(d)
+    K = rng.standard_normal((Nk, d))
+    V = rng.standard_normal((Nk, d))
+    keep_b, O_b = _brute_forward(Q, K, V, Bq, Bk, tau)
+    O, z, keep, _ = orc.forward_head(Q, K, V, Bq, Bk, tau)
+    assert (keep == keep_b).all()
+    assert np.abs(O - O_b).max() < 1e-12
+
+
+@pytest.mark.parametrize("tau", [0.1, 1.0])
+def test_bottom_right_aligned_chunk_is_the_last_rows_of_the_full_problem(tau):
+    """With an offset that is a multiple of both block sizes, the chunk's
+    query blocks are the full problem's last query blocks: same decisions,
+    outputs and, with dO zero on the other rows, the same gradients."""
+    rng = np.random.default_rng(77)
+    Nk, off, d, B = 48, 16, 5, 8
+    Q = rng.standard_normal((Nk, d)) * 5 / math.sqrt(d)
+    K = rng.standard_normal((Nk, d))
+    V = rng.standard_normal((Nk, d))
+    dO = rng.standard_normal((Nk, d))
+    dO[:off] = 0.0
+    O_f, z_f, keep_f, _ = orc.forward_head(Q, K, V, B, B, tau)
+    O_c, z_c, keep_c, _ = orc.forward_head(Q[off:], K, V, B, B, tau)
+    assert np.abs(O_c - O_f[off:]).max() < 1e-12 and np.abs(z_c - z_f[off:]).max() < 1e-12
+    assert (keep_c == keep_f[off // B:]).all()
+    assert keep_c.sum() < keep_c.size             # the case exercises skipping
+    dQ_f, dK_f, dV_f, bk_f, _ = orc.backward_head(Q, K, V, O_f, dO, z_f, B, B, tau, keep_f)
+    dQ_c, dK_c, dV_c, bk_c, _ = orc.backward_head(Q[off:], K, V, O_c, dO[off:], z_c, B, B, tau, keep_c)
+    assert np.abs(dQ_c - dQ_f[off:]).max() < 1e-12
+    assert np.abs(dK_c - dK_f).max() < 1e-12 and np.abs(dV_c - dV_f).max() < 1e-12
+    assert (bk_c == bk_f[off // B:]).all()
+
+
+def test_bottom_right_single_query_is_decoding():
+    rng = np.random.default_rng(9)
+    Nk, d, Bk = 45, 6, 8
+    Q = rng.standard_normal((1, d)) * 3 / math.sqrt(d)
+    K = rng.standard_normal((Nk, d))
+    V = rng.standard_normal((Nk, d))
+    for tau in (0.0, 0.2, 1.5):
+        O, z, keep, _ = orc.forward_head(Q, K, V, 4, Bk, tau)
+        Od, zd, kd, _, _ = orc.decode_head(Q[0], K, V, Bk, tau, 1)
+        assert np.allclose(Od, O[0], atol=1e-14) and abs(zd - z[0]) < 1e-14
+        assert (kd == keep[0]).all()
