@@ -68,7 +68,10 @@ enum { MALA_BF16 = 0, MALA_FP32 = 1 };
 
 /* masking mode of mala_fwd */
 enum {
-  MALA_CAUSAL = 0,  /* N_q = N_k, key k legal for row q iff k <= q, L_q = q + 1 */
+  MALA_CAUSAL = 0,  /* N_q <= N_k, bottom-right aligned: query q sits at position
+                       p_q = q + N_k - N_q, key k is legal iff k <= p_q, L_q = p_q + 1
+                       (N_q = N_k: L_q = q + 1; a chunk of queries appended to a
+                       context of N_k - N_q keys otherwise) */
   MALA_DECODE = 1   /* reserved for mala_fwd: single-token decoding uses mala_decode */
 };
 
@@ -132,7 +135,9 @@ MALA_API int mala_fwd(const mala_fwd_args* args, void* workspace, size_t workspa
  * argument of the same section this selects the same tiles up to rounding).
  * NULL visits every legal tile. bwd_keep_mask (output, optional): same
  * layout, bits of tiles the backward retained. dq, dk, dv are fully
- * overwritten. Supported: MALA_BF16, d = 128, B_q = B_k = 128.
+ * overwritten. Supported: MALA_BF16, d = 128, B_q = B_k = 128, causal with
+ * N_q <= N_k bottom-right aligned as for mala_fwd (key rows that no query
+ * sees get dK = dV = 0).
  */
 typedef struct {
   const void* q;

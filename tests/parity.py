@@ -94,7 +94,8 @@ def check_fwd(q, k, v, o, lse, keep_words, tau, B_q, B_k, samples=None, rep=None
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
     G = Hq // Hkv
-    nQB, nKB = orc.num_blocks(N, B_q), orc.num_blocks(N, B_k)
+    off = k.shape[1] - N                          # bottom-right alignment when N_q < N_k
+    nQB, nKB = orc.num_blocks(N, B_q), orc.num_blocks(k.shape[1], B_k)
     keep = mala.unpack_mask(keep_words, nKB)
     o64 = None
     if samples is None:
@@ -108,8 +109,8 @@ def check_fwd(q, k, v, o, lse, keep_words, tau, B_q, B_k, samples=None, rep=None
         Oh = f64(o[b, :, h])
         for i in blocks:
             q0, q1 = i * B_q, min((i + 1) * B_q, N)
-            pos = np.arange(q0, q1)
-            tiles = orc.causal_tiles(q1 - 1, B_k, nKB)
+            pos = np.arange(q0, q1) + off
+            tiles = orc.causal_tiles(q1 - 1 + off, B_k, nKB)
             check_fwd_block(Qh[q0:q1], Kh, Vh, pos, tiles, B_k, tau, keep[b, h, i], Oh[q0:q1],
                             lse_c[b, h, q0:q1], rep, f"fwd b={b} h={h} i={i}")
     return rep
@@ -175,14 +176,15 @@ def oracle_forward_replaying(q64, k64, v64, b, h, G, blocks, gpu_keep_bh, B_q, B
     O [N, d] and z [N] arrays (NaN outside the blocks)."""
     Q, K, V = q64[b, :, h], k64[b, :, h // G], v64[b, :, h // G]
     N = Q.shape[0]
-    nKB = orc.num_blocks(N, B_k)
+    off = K.shape[0] - N
+    nKB = orc.num_blocks(K.shape[0], B_k)
     O = np.full((N, V.shape[1]), np.nan)
     z = np.full(N, np.nan)
     for i in blocks:
         q0, q1 = i * B_q, min((i + 1) * B_q, N)
-        tiles = orc.causal_tiles(q1 - 1, B_k, nKB)
+        tiles = orc.causal_tiles(q1 - 1 + off, B_k, nKB)
         gdec = {j: bool(gpu_keep_bh[i, j]) for j in tiles}
-        st = orc.forward_block(Q[q0:q1], np.arange(q0, q1), K, V, B_k, tau, tiles, replay=gdec)
+        st = orc.forward_block(Q[q0:q1], np.arange(q0, q1) + off, K, V, B_k, tau, tiles, replay=gdec)
         for j in tiles:
             mj = st["margin"][j]
             if gdec[j] != (mj <= 0.0):
@@ -212,7 +214,9 @@ def check_bwd_blocks(q, k, v, do, fwd_keep_words, bwd_keep_words, dq, dk, dv, ta
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
     G = Hq // Hkv
-    nQB, nKB = orc.num_blocks(N, B_q), orc.num_blocks(N, B_k)
+    Nk = k.shape[1]
+    off = Nk - N                                  # bottom-right alignment when N_q < N_k
+    nQB, nKB = orc.num_blocks(N, B_q), orc.num_blocks(Nk, B_k)
     fkeep = mala.unpack_mask(fwd_keep_words, nKB)
     bkeep = mala.unpack_mask(bwd_keep_words, nKB) if bwd_keep_words is not None else None
     q64, k64, v64, do64 = f64(q), f64(k), f64(v), f64(do)
@@ -253,11 +257,12 @@ def check_bwd_blocks(q, k, v, do, fwd_keep_words, bwd_keep_words, dq, dk, dv, ta
                         f"bwd b={b} h={h} tile ({i},{j}): margin {bm_ref[i, j]:.3e}"
 
     for (b, hk, j) in kv_samples:
-        k0, k1 = j * B_k, min((j + 1) * B_k, N)
+        k0, k1 = j * B_k, min((j + 1) * B_k, Nk)
         dK = np.zeros((k1 - k0, d))
         dV = np.zeros((k1 - k0, d))
+        i_first = max(0, k0 - off) // B_q
         for h in range(hk * G, (hk + 1) * G):
-            blocks = [i for i in range(j, nQB) if fkeep[b, h, i, j]]
+            blocks = [i for i in range(i_first, nQB) if fkeep[b, h, i, j]]
             if not blocks:
                 continue
             O, z = fwd_rows(b, h, blocks)
@@ -284,7 +289,7 @@ def check_bwd_blocks(q, k, v, do, fwd_keep_words, bwd_keep_words, dq, dk, dv, ta
         dQh, _, _, bk_ref, bm_ref = orc.backward_head(
             q64[b, :, h], k64[b, :, h // G], v64[b, :, h // G], O, do64[b, :, h], z, B_q, B_k, tau,
             fkeep[b, h], qblocks=[i])
-        check_bmask(b, h, bk_ref, bm_ref, [i], range(0, i + 1))
+        check_bmask(b, h, bk_ref, bm_ref, [i], range(0, min(nKB, (q1 - 1 + off) // B_k + 1)))
         got, ref = dq64[b, q0:q1, h], dQh[q0:q1]
         assert np.isfinite(got).all(), f"dQ b={b} h={h} i={i}: non-finite"
         if np.linalg.norm(ref) == 0.0:

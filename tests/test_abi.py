@@ -107,7 +107,7 @@ def _fwd_args(**kw):
     (dict(q=0x10008), mala.MALA_ERR_INVALID_ARG),           # misaligned base
     (dict(q_stride=mala._i64x3(256 * 4 * 128, 4 * 128 + 3, 128)), mala.MALA_ERR_INVALID_ARG),
     (dict(head_dim=96), mala.MALA_ERR_UNSUPPORTED),
-    (dict(seqlen_k=128), mala.MALA_ERR_UNSUPPORTED),         # causal needs Nq == Nk
+    (dict(seqlen_k=128), mala.MALA_ERR_UNSUPPORTED),         # causal needs Nq <= Nk
     (dict(block_q=48), mala.MALA_ERR_UNSUPPORTED),
     (dict(mode=mala.MALA_DECODE), mala.MALA_ERR_UNSUPPORTED),
     (dict(dtype=7), mala.MALA_ERR_INVALID_ARG),

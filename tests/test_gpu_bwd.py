@@ -151,3 +151,37 @@ def test_train_8k_full_size_sampled():
     fm = mala.unpack_mask(keep, nQB)
     bm = mala.unpack_mask(bkeep, nQB)
     assert s[0] == fm.sum() and s[1] == bm.sum()
+
+
+# ------------------------------------------- bottom-right causal alignment
+
+def _chunk(B, Nq, Nk, Hq, Hkv, seed):
+    g = torch.Generator().manual_seed(seed)
+    d = 128
+    return {"q": (torch.randn(B, Nk, Hq, d, generator=g) * 3 / math.sqrt(d))[:, Nk - Nq:].bfloat16().to(DEV),
+            "k": torch.randn(B, Nk, Hkv, d, generator=g).bfloat16().to(DEV),
+            "v": torch.randn(B, Nk, Hkv, d, generator=g).bfloat16().to(DEV),
+            "do": torch.randn(B, Nq, Hq, d, generator=g).bfloat16().to(DEV)}
+
+
+@pytest.mark.parametrize("Nq,Nk", [(1, 300), (100, 164), (128, 384), (200, 456), (129, 1000)])
+def test_bottom_right_chunk_backward(Nq, Nk):
+    t = _chunk(2, Nq, Nk, 4, 2, seed=Nq + 3 * Nk)
+    o, lse, keep, dq, dk, dv, bkeep = _fwd_bwd(t, 0.3)
+    check_bwd_blocks(t["q"], t["k"], t["v"], t["do"], keep, bkeep, dq, dk, dv, 0.3)
+
+
+@pytest.mark.parametrize("pure", [False, True])
+def test_bottom_right_chunk_backward_recipe_skips(pure):
+    t = _run(synth.WORKLOADS["train_8k"], batch=1, seqlen=1024)
+    Nq = 320
+    t["q"] = t["q"][:, 1024 - Nq:]
+    t["do"] = t["do"][:, 1024 - Nq:]
+    o, lse, keep, dq, dk, dv, bkeep = _fwd_bwd(t, 1.0, pure=pure)
+    fm = mala.unpack_mask(keep, 8)
+    bm = mala.unpack_mask(bkeep, 8)
+    legal = sum(min((i * 128 + 127 + 1024 - Nq) // 128, 7) + 1 for i in range(3))
+    assert bm.sum() < legal * 16                    # the sharp heads skip tiles
+    if not pure:
+        assert not (bm & ~fm).any()                 # mask replay visits forward-kept tiles only
+    check_bwd_blocks(t["q"], t["k"], t["v"], t["do"], keep, bkeep if not pure else None, dq, dk, dv, 1.0)

@@ -7,7 +7,7 @@ import torch
 
 from oracle import mala_oracle as orc
 from tile_skipping_causal_b200 import mala, synth
-from tests.parity import FwdReport, assert_close, check_fwd, f64
+from tests.parity import FwdReport, assert_close, check_decode, check_fwd, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -165,3 +165,62 @@ def test_stats_count_kept_tiles():
     assert s[0] == 16 * 8 * 9 // 2
     assert s[1] == m.sum()
     assert s[2] == m.sum() * 128 * 128
+
+
+# ------------------------------------------- bottom-right causal alignment
+# A chunk of N_q queries appended to a context of N_k - N_q keys: query q sits
+# at position q + N_k - N_q. The chunk is the last N_q query rows of a longer
+# seeded problem (a strided view, as a chunked-prefill caller would pass it).
+
+@pytest.mark.parametrize("Nq,Nk", [(1, 700), (100, 164), (128, 384), (200, 456), (300, 301), (129, 1000)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_bottom_right_chunk_gqa(Nq, Nk, d):
+    t = _random_bf16(2, Nk, 4, 2, d, seed=Nq * 7 + Nk + d)
+    q = t["q"][:, Nk - Nq:]
+    o, lse, keep = mala.mala_fwd(q, t["k"], t["v"], 0.3, 128, 128)
+    mala.check_device_error()
+    assert keep.shape[-1] == mala.mask_words(-(-Nk // 128))
+    check_fwd(q, t["k"], t["v"], o, lse, keep, 0.3, 128, 128)
+
+
+@pytest.mark.parametrize("tau", [0.1, 1.0])
+def test_bottom_right_chunk_recipe_skips(tau):
+    t = _run(synth.WORKLOADS["prefill_4k"], batch=1, seqlen=1024)
+    q = t["q"][:, 1024 - 320:]
+    stats = torch.zeros(4, dtype=torch.int64, device=DEV)
+    o, lse, keep = mala.mala_fwd(q, t["k"], t["v"], tau, 128, 128, stats=stats)
+    mala.check_device_error()
+    rep = check_fwd(q, t["k"], t["v"], o, lse, keep, tau, 128, 128)
+    tested, kept = stats[0].item(), stats[1].item()
+    assert tested == rep.tiles and kept == rep.kept
+    if tau == 1.0:
+        assert kept < tested                      # the sharp heads skip tiles
+
+
+def test_bottom_right_cuda_core_path():
+    g = torch.Generator().manual_seed(3)
+    B, Nk, Nq, H, d = 1, 333, 90, 2, 64
+    q = (torch.randn(B, Nk, H, d, generator=g) * 3 / math.sqrt(d))[:, Nk - Nq:].to(DEV)
+    k = torch.randn(B, Nk, H, d, generator=g).to(DEV)
+    v = torch.randn(B, Nk, H, d, generator=g).to(DEV)
+    o, lse, keep = mala.mala_fwd(q, k, v, 0.2, 64, 64)
+    mala.check_device_error()
+    check_fwd(q, k, v, o, lse, keep, 0.2, 64, 64)
+
+
+def test_bottom_right_single_query_matches_decode():
+    """N_q = 1 is the decoding case (L_0 = N_k): the prefill kernel on a
+    one-row chunk and the decode kernel without splits agree."""
+    g = torch.Generator().manual_seed(11)
+    B, Nk, Hq, Hkv, d = 2, 1000, 8, 2, 128
+    q = (torch.randn(B, 1, Hq, d, generator=g) * 3 / math.sqrt(d)).bfloat16().to(DEV)
+    k = torch.randn(B, Nk, Hkv, d, generator=g).bfloat16().to(DEV)
+    v = torch.randn(B, Nk, Hkv, d, generator=g).bfloat16().to(DEV)
+    o, lse, keep = mala.mala_fwd(q, k, v, 0.05, 128, 128)
+    od, lsed, keepd, P = mala.mala_decode(q, k, v, 0.05, 128, 1)
+    mala.check_device_error()
+    assert P == 1
+    check_fwd(q, k, v, o, lse, keep, 0.05, 128, 128)
+    check_decode(q, k, v, od, lsed, keepd, 0.05, P)
+    assert_close(f64(o), f64(od), "O fwd vs decode")
+    assert_close(lse.cpu().numpy().reshape(B, Hq), lsed.cpu().numpy(), "LSE fwd vs decode")

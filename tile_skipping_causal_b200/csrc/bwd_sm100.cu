@@ -128,8 +128,11 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         tma_load_4d(sK + c * kChunk, &p.tm_k, &bars[kKVFull], c * 64, hk, j * kB, b);
         tma_load_4d(sV + c * kChunk, &p.tm_v, &bars[kKVFull], c * 64, hk, j * kB, b);
       }
-      // scan state of the next visited tile (group head g, query block i)
-      int sg = 0, si = j;
+      // scan state of the next visited tile (group head g, query block i);
+      // the first query block with a row at or after key block j's first key
+      // (query q sits at position q + q_off)
+      const int i_first = max(0, j * kB - p.q_off) / kB;
+      int sg = 0, si = i_first;
       auto next_tile = [&](int& h_out, int& i_out) -> bool {
         while (sg < G) {
           const int h = p.group_heads[hk][sg];
@@ -143,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
             }
           }
           ++sg;
-          si = j;
+          si = i_first;
         }
         return false;
       };
@@ -358,11 +361,13 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       const float4* zl2_4 = reinterpret_cast<const float4*>(sStats + st * 384 + c0);
       const float4* thr_4 = reinterpret_cast<const float4*>(sStats + st * 384 + 128 + c0);
       const float4* dv_4 = reinterpret_cast<const float4*>(sStats + st * 384 + 256 + c0);
-      // test over this half of the S^T row. Legal entries: query column
-      // c >= key row r on the diagonal tile; padded query rows carry an
-      // infinite threshold and never count
+      // test over this half of the S^T row. Legal entries: query columns
+      // x >= lim (at or after the key's position); padded query rows carry
+      // an infinite threshold and never count
       const bool oks = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], n & 1, abort_flag, p.err, wait_tag(0, kSFull, n)));
-      const int lim = ((i == j) ? r : 0) - c0;  // first legal column of this half
+      // first legal column of this half for key row r: query column c is at
+      // position i * 128 + c + q_off and sees key j * 128 + r iff that is >= it
+      const int lim = (j * kB + r) - (i * kB + p.q_off) - c0;
       uint32_t sr[2][32];
       if (oks) {
         tc_fence_after();
@@ -503,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
           tmem_ld32(base + lane_addr + c0 + c * 32, rr);
           tmem_ld_wait(rr);
           reg_fence(rr);
-          if (krow < p.N) {
+          if (krow < p.Nk) {
             uint32_t pk[16];
 #pragma unroll
             for (int x = 0; x < 32; x += 2)
@@ -563,7 +568,7 @@ __global__ void __launch_bounds__(128) mala_bwd_pre_kernel(const __grid_constant
     const float z = p.lse[static_cast<int64_t>(bh) * p.N + q];
     p.Dv[row] = acc;
     p.zl2[row] = z * kLog2e;
-    p.t2[row] = z + p.log_tau - logf(static_cast<float>(q + 1));
+    p.t2[row] = z + p.log_tau - logf(static_cast<float>(q + p.q_off + 1));
   } else {
     p.Dv[row] = 0.0f;
     p.zl2[row] = INFINITY;

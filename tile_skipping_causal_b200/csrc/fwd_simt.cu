@@ -48,8 +48,9 @@ __global__ void __launch_bounds__(128) mala_fwd_simt_kernel(const FwdSimtParams 
   const int q0 = i * BQ;
   const int q = q0 + r;
   const bool valid = q < p.N;
+  const int qa = q + p.q_off;                     // position of the row (bottom-right alignment)
   const int last_row = min(q0 + BQ - 1, p.N - 1);
-  const int j_diag = min(last_row / BK, p.nKB - 1);
+  const int j_diag = min((last_row + p.q_off) / BK, p.nKB - 1);
 
   const T* Q = reinterpret_cast<const T*>(p.q);
   const T* K = reinterpret_cast<const T*>(p.k);
@@ -62,7 +63,7 @@ __global__ void __launch_bounds__(128) mala_fwd_simt_kernel(const FwdSimtParams 
     qr[x] = valid ? to_f32(Q[b * p.q_sb + static_cast<int64_t>(q) * p.q_sn + h * p.q_sh + x]) : 0.0f;
     acc[x] = 0.0f;
   }
-  const float thr = p.log_tau - logf(static_cast<float>(q + 1));   // log(tau / L_q)
+  const float thr = p.log_tau - logf(static_cast<float>(qa + 1));   // log(tau / L_q)
   float m = -INFINITY, l = 0.0f;
   uint32_t mask_word = 0;
   int kept_tiles = 0;
@@ -75,10 +76,10 @@ __global__ void __launch_bounds__(128) mala_fwd_simt_kernel(const FwdSimtParams 
     __syncthreads();
     for (int e = r; e < BK * D; e += BQ) {
       const int c = e / D, x = e % D, k = k0 + c;
-      sK[e] = (k < p.N) ? to_f32(K[b * p.k_sb + static_cast<int64_t>(k) * p.k_sn + hk * p.k_sh + x]) : 0.0f;
+      sK[e] = (k < p.Nk) ? to_f32(K[b * p.k_sb + static_cast<int64_t>(k) * p.k_sn + hk * p.k_sh + x]) : 0.0f;
     }
     __syncthreads();
-    const int lim = q - k0;                       // legal columns: c <= lim
+    const int lim = qa - k0;                      // legal columns: c <= lim
     const bool has_key = valid && lim >= 0;
     float rmax = -INFINITY;
     for (int c = 0; c < BK; ++c) {
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(128) mala_fwd_simt_kernel(const FwdSimtParams 
     if (!keep) continue;
     for (int e = r; e < BK * D; e += BQ) {
       const int c = e / D, x = e % D, k = k0 + c;
-      sV[e] = (k < p.N) ? to_f32(V[b * p.v_sb + static_cast<int64_t>(k) * p.v_sn + hk * p.v_sh + x]) : 0.0f;
+      sV[e] = (k < p.Nk) ? to_f32(V[b * p.v_sb + static_cast<int64_t>(k) * p.v_sn + hk * p.v_sh + x]) : 0.0f;
     }
     __syncthreads();
     if (has_key) {

@@ -131,7 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
   const int hk = p.kv_of_q[h];
   const int q0 = i * kBQ;
   const int last_row = min(q0 + kBQ - 1, p.N - 1);
-  const int j_diag = min(last_row / kBK, p.nKB - 1);
+  // bottom-right alignment: query row q sits at position q + q_off
+  const int j_diag = min((last_row + p.q_off) / kBK, p.nKB - 1);
   const int T = j_diag + 1;         // tile t visits key block j = j_diag - t
 
   if (tid == 0) {
@@ -287,8 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
     const int c0 = g * 64;
     const int q = q0 + r;
     const bool valid = q < p.N;
+    const int qa = q + p.q_off;                 // the row's position: keys k <= qa are legal
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const float thr2 = p.log2_tau - log2f(static_cast<float>(q + 1));   // log2(tau / L_q)
+    const float thr2 = p.log2_tau - log2f(static_cast<float>(qa + 1));   // log2(tau / L_q)
     float m2 = -INFINITY;                    // reference maximum, log2 units
     float l = 0.0f;                          // sum of 2^(s log2e - m2) over retained keys
     int kc = 0;
@@ -319,12 +321,13 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       reg_fence(sr[0]);
       reg_fence(sr[1]);
 
-      // causal mask: key k = j*128 + c is legal iff k <= q; this group's
-      // columns are c = c0 + x. Only the diagonal tile (t = 0) has illegal
-      // keys: every earlier key block lies below the block's first row.
-      const bool has_key = valid && q >= j * kBK;
-      if (t == 0) {
-        const int lim = q - j * kBK - c0;     // largest legal x
+      // causal mask: key k = j*128 + c is legal iff k <= qa; this group's
+      // columns are c = c0 + x. Only tiles whose last key lies beyond the
+      // block's first row position can hold illegal keys (the diagonal
+      // tile, and the one before it when q_off is not a multiple of 128).
+      const bool has_key = valid && qa >= j * kBK;
+      if (j * kBK + kBK - 1 > q0 + p.q_off) {
+        const int lim = qa - j * kBK - c0;    // largest legal x
 #pragma unroll
         for (int x = 0; x < 64; ++x)
           if (x > lim) sr[x >> 5][x & 31] = __float_as_uint(-INFINITY);

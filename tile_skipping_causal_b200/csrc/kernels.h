@@ -21,7 +21,8 @@ struct FwdTcParams {
   int64_t* stats;
   int* err;             // library device error block int[4]
   int64_t o_sb, o_sn, o_sh;
-  int B, Hq, Hkv, N;
+  int B, Hq, Hkv, N;    // N = N_q
+  int Nk, q_off;        // N_k >= N_q; query q sits at position q + q_off (q_off = N_k - N_q)
   int nQB, nKB, mask_words;
   float log2_tau;       // log2(tau): -inf for tau = 0, +inf for tau = inf
   uint8_t kv_of_q[kMaxHeads];
@@ -40,7 +41,8 @@ struct FwdSimtParams {
   uint32_t* keep_mask;
   int64_t* stats;
   int64_t q_sb, q_sn, q_sh, k_sb, k_sn, k_sh, v_sb, v_sn, v_sh, o_sb, o_sn, o_sh;
-  int B, Hq, Hkv, N;
+  int B, Hq, Hkv, N;    // N = N_q
+  int Nk, q_off;        // N_k >= N_q; query q sits at position q + q_off
   int BQ, BK;
   int nQB, nKB, mask_words;
   float log_tau;        // natural log of tau (+-inf allowed)
@@ -75,7 +77,7 @@ struct DecodeParams {
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
 size_t decode_smem_bytes();
 
-// Backward (bf16, d = 128, B_q = B_k = 128, N_q = N_k).
+// Backward (bf16, d = 128, B_q = B_k = 128, N_q <= N_k bottom-right aligned).
 struct BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;   // 4-D maps, box {64, 1, 128, 1}, 128B swizzle
   const float* zl2;        // [B, Hq, Npad] z log2e
@@ -89,7 +91,8 @@ struct BwdParams {
   int64_t* stats;
   int* err;
   int64_t dk_sb, dk_sn, dk_sh, dv_sb, dv_sn, dv_sh;
-  int B, Hq, Hkv, N, Npad, nQB, nKB, mask_words;
+  int B, Hq, Hkv, N, Npad, nQB, nKB, mask_words;   // N = N_q, Npad = nQB * 128
+  int Nk, q_off;           // N_k >= N_q; query q sits at position q + q_off
   uint8_t group_size[kMaxKvHeads];
   uint8_t group_heads[kMaxKvHeads][kMaxGroup];
 };
@@ -104,7 +107,8 @@ struct BwdAuxParams {      // pre-pass and dQ conversion
   float* dq_acc;
   void* dq;
   int64_t o_sb, o_sn, o_sh, do_sb, do_sn, do_sh, dq_sb, dq_sn, dq_sh;
-  int B, Hq, N, Npad, nQB;
+  int B, Hq, N, Npad, nQB;   // N = N_q
+  int q_off;                 // query q sits at position q + q_off: L_q = q + q_off + 1
   float log_tau;
 };
 

@@ -181,9 +181,9 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
   if (a->mode != MALA_CAUSAL)
     return fail(MALA_ERR_UNSUPPORTED, "mala_fwd supports MALA_CAUSAL; use mala_decode for decoding");
   if (a->seqlen_q <= 0 || a->seqlen_k <= 0) return fail(MALA_ERR_INVALID_ARG, "sequence lengths must be positive");
-  if (a->seqlen_q != a->seqlen_k)
-    return fail(MALA_ERR_UNSUPPORTED, "causal mode needs seqlen_q == seqlen_k");
-  if (a->seqlen_q > (1 << 30)) return fail(MALA_ERR_UNSUPPORTED, "sequence too long");
+  if (a->seqlen_q > a->seqlen_k)
+    return fail(MALA_ERR_UNSUPPORTED, "causal mode needs seqlen_q <= seqlen_k (bottom-right alignment)");
+  if (a->seqlen_k > (1 << 30)) return fail(MALA_ERR_UNSUPPORTED, "sequence too long");
   if (!block_ok(a->block_q) || !block_ok(a->block_k))
     return fail(MALA_ERR_UNSUPPORTED, "block sizes must be in {16, 32, 64, 128}");
   if (!a->lse) return fail(MALA_ERR_INVALID_ARG, "lse is NULL");
@@ -197,8 +197,9 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
   if (a->stats && (reinterpret_cast<uintptr_t>(a->stats) & 7u) != 0)
     return fail(MALA_ERR_INVALID_ARG, "stats misaligned");
   const int64_t N = a->seqlen_q;
+  const int64_t Nk = a->seqlen_k;
   const int nQB = static_cast<int>((N + a->block_q - 1) / a->block_q);
-  const int nKB = static_cast<int>((N + a->block_k - 1) / a->block_k);
+  const int nKB = static_cast<int>((Nk + a->block_k - 1) / a->block_k);
   const int mask_words = (nKB + 31) / 32;
   if ((double)a->batch * a->heads_q * nQB > 2147483647.0) return fail(MALA_ERR_UNSUPPORTED, "grid too large");
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
@@ -209,8 +210,8 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
     memset(&p, 0, sizeof(p));
     if ((rc = head_map(a->q_to_kv, a->heads_q, a->heads_kv, p.kv_of_q))) return rc;
     if ((rc = make_map_bf16(&p.tm_q, a->q, a->batch, N, a->heads_q, d, a->q_stride, 128))) return rc;
-    if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, N, a->heads_kv, d, a->k_stride, 128))) return rc;
-    if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, N, a->heads_kv, d, a->v_stride, 128))) return rc;
+    if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, Nk, a->heads_kv, d, a->k_stride, 128))) return rc;
+    if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, Nk, a->heads_kv, d, a->v_stride, 128))) return rc;
     p.err = device_error_ptr();
     if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
     p.o = a->o;
@@ -224,6 +225,8 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
     p.Hq = static_cast<int>(a->heads_q);
     p.Hkv = static_cast<int>(a->heads_kv);
     p.N = static_cast<int>(N);
+    p.Nk = static_cast<int>(Nk);
+    p.q_off = static_cast<int>(Nk - N);
     p.nQB = nQB;
     p.nKB = nKB;
     p.mask_words = mask_words;
@@ -250,6 +253,8 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
   p.Hq = static_cast<int>(a->heads_q);
   p.Hkv = static_cast<int>(a->heads_kv);
   p.N = static_cast<int>(N);
+  p.Nk = static_cast<int>(Nk);
+  p.q_off = static_cast<int>(Nk - N);
   p.BQ = a->block_q;
   p.BK = a->block_k;
   p.nQB = nQB;
@@ -272,8 +277,9 @@ int bwd_check(const mala_bwd_args* a) {
   if (a->head_dim != 128) return fail(MALA_ERR_UNSUPPORTED, "backward supports head_dim 128 only");
   if (a->block_q != 128 || a->block_k != 128) return fail(MALA_ERR_UNSUPPORTED, "backward supports 128 x 128 tiles only");
   if (a->seqlen_q <= 0 || a->seqlen_k <= 0) return fail(MALA_ERR_INVALID_ARG, "sequence lengths must be positive");
-  if (a->seqlen_q != a->seqlen_k) return fail(MALA_ERR_UNSUPPORTED, "causal backward needs seqlen_q == seqlen_k");
-  if (a->seqlen_q > (1 << 30)) return fail(MALA_ERR_UNSUPPORTED, "sequence too long");
+  if (a->seqlen_q > a->seqlen_k)
+    return fail(MALA_ERR_UNSUPPORTED, "causal backward needs seqlen_q <= seqlen_k (bottom-right alignment)");
+  if (a->seqlen_k > (1 << 30)) return fail(MALA_ERR_UNSUPPORTED, "sequence too long");
   if (a->heads_kv > mala::kMaxKvHeads) return fail(MALA_ERR_UNSUPPORTED, "heads_kv > %d", mala::kMaxKvHeads);
   if (!a->lse) return fail(MALA_ERR_INVALID_ARG, "lse is NULL");
   if ((rc = check_tensor("q", a->q, a->q_stride, 2, 128, a->heads_q))) return rc;
@@ -310,7 +316,9 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
   if (!workspace || ws_bytes < need) return fail(MALA_ERR_WORKSPACE, "backward workspace of %zu bytes needed", need);
   if (!aligned16(workspace)) return fail(MALA_ERR_INVALID_ARG, "workspace misaligned");
   const int N = static_cast<int>(a->seqlen_q);
+  const int Nk = static_cast<int>(a->seqlen_k);
   const int nQB = (N + 127) / 128;
+  const int nKB = (Nk + 127) / 128;
   const int Npad = nQB * 128;
   const size_t rows = static_cast<size_t>(a->batch) * a->heads_q * Npad;
 
@@ -325,8 +333,8 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
     p.group_heads[hk][p.group_size[hk]++] = static_cast<uint8_t>(h);
   }
   if ((rc = make_map_bf16(&p.tm_q, a->q, a->batch, N, a->heads_q, 128, a->q_stride, 128))) return rc;
-  if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, N, a->heads_kv, 128, a->k_stride, 128))) return rc;
-  if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, N, a->heads_kv, 128, a->v_stride, 128))) return rc;
+  if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, Nk, a->heads_kv, 128, a->k_stride, 128))) return rc;
+  if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, Nk, a->heads_kv, 128, a->v_stride, 128))) return rc;
   if ((rc = make_map_bf16(&p.tm_do, a->dout, a->batch, N, a->heads_q, 128, a->do_stride, 128))) return rc;
   float* ws = static_cast<float*>(workspace);
   p.zl2 = ws;
@@ -346,10 +354,12 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
   p.Hq = static_cast<int>(a->heads_q);
   p.Hkv = static_cast<int>(a->heads_kv);
   p.N = N;
+  p.Nk = Nk;
+  p.q_off = Nk - N;
   p.Npad = Npad;
   p.nQB = nQB;
-  p.nKB = nQB;
-  p.mask_words = (nQB + 31) / 32;
+  p.nKB = nKB;
+  p.mask_words = (nKB + 31) / 32;
 
   mala::BwdAuxParams x;
   memset(&x, 0, sizeof(x));
@@ -369,6 +379,7 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
   x.N = N;
   x.Npad = Npad;
   x.nQB = nQB;
+  x.q_off = Nk - N;
   x.log_tau = a->tau == 0.0f ? -INFINITY : logf(a->tau);
 
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
