@@ -277,6 +277,7 @@ def run_mala(args):
     del dense
 
     peaks = _peaks()
+    chunk = bench_chunk(args, q, k, v, stream, peaks)
     dec = None if args.no_decode else bench_decode(args, dev, stream, peaks)
     kern_f = statistics.mean(fwd_times)
     kern_b = statistics.mean(bwd_times)
@@ -322,6 +323,7 @@ def run_mala(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
+    res["chunked_prefill"] = chunk
     if dec is not None:
         res["decode"] = dec
     if rank == 0 and not args.no_cpu_baseline and world == 1:
@@ -331,6 +333,39 @@ def run_mala(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(res), flush=True)
+
+
+def bench_chunk(args, q, k, v, stream, peaks, chunk: int = 4096):
+    """Chunked prefill: the forward of the last ``chunk`` queries of the
+    workload against all of its keys (bottom-right causal alignment, query q
+    at position q + N_k - N_q), on the same inputs. Executed FLOPs as for
+    the full forward: every tested tile pays QK^T, every retained one PV."""
+    import torch
+    from tile_skipping_causal_b200 import mala
+
+    Nk = k.shape[1]
+    qc = q[:, Nk - chunk:]
+    stats = torch.zeros(4, dtype=torch.int64, device=q.device)
+    o, lse, keep = mala.mala_fwd(qc, k, v, TAU, TILE, TILE, stats=stats)
+    mala.check_device_error()
+    tested, kept = (int(x) for x in stats.cpu().tolist()[:2])
+    for _ in range(max(3, args.warmup)):
+        mala.mala_fwd(qc, k, v, TAU, TILE, TILE, o=o, lse=lse, keep_mask=keep)
+    torch.cuda.synchronize()
+    n = max(5, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        mala.mala_fwd(qc, k, v, TAU, TILE, TILE, o=o, lse=lse, keep_mask=keep)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    mala.check_device_error()
+    t = e0.elapsed_time(e1) / 1e3 / n
+    flops = tile_flops(q.shape[3]) * (tested + kept)
+    peak = peaks["bf16_tflops_sustained"]
+    return {"seqlen_q": chunk, "seqlen_k": Nk, "tau": TAU, "ms": t * 1e3,
+            "tokens_per_s": q.shape[0] * chunk / t, "tiles_tested": tested, "tiles_kept": kept,
+            "tflops_executed": flops / t / 1e12, "frac_of_peak": flops / t / 1e12 / peak}
 
 
 def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072):

@@ -114,7 +114,21 @@ typedef struct {
   int32_t dtype;
   int32_t mode;
   int64_t* stats;               /* device int64[4] or NULL */
+  /* Packed variable-length sequences (NULL = fixed lengths). HOST arrays of
+   * batch + 1 ascending offsets, cu_seqlens_q[0] = cu_seqlens_k[0] = 0:
+   * sequence s owns query rows [cu_seqlens_q[s], cu_seqlens_q[s+1]) and key
+   * rows [cu_seqlens_k[s], cu_seqlens_k[s+1]), each bottom-right aligned on
+   * its own (N_q,s <= N_k,s). q, o are then [1, total_q, H_q, d] and k, v
+   * [1, total_k, H_kv, d] (stride[0] unused); seqlen_q / seqlen_k give the
+   * totals; lse is [H_q, total_q]; keep_mask is [H_q, QB, ceil(KB/32)] with
+   * QB = sum_s ceil(N_q,s / B_q) (sequence s's blocks after those of the
+   * earlier sequences) and KB = max_s ceil(N_k,s / B_k). Tensor-core path
+   * only (bf16, 128 x 128 tiles); at most MALA_MAX_SEQS sequences. */
+  const int32_t* cu_seqlens_q;
+  const int32_t* cu_seqlens_k;
 } mala_fwd_args;
+
+#define MALA_MAX_SEQS 128
 
 MALA_API size_t mala_fwd_workspace_size(const mala_fwd_args* args);
 MALA_API int mala_fwd(const mala_fwd_args* args, void* workspace, size_t workspace_bytes,
@@ -165,6 +179,11 @@ typedef struct {
   float tau;
   int32_t dtype;
   int64_t* stats;               /* device int64[4]: tiles tested, retained, slots, reserved */
+  /* Packed variable-length sequences, as for mala_fwd (NULL = fixed
+   * lengths); dout and dq follow q's packed layout, dk and dv k's; lse and
+   * the masks use mala_fwd's packed layouts. */
+  const int32_t* cu_seqlens_q;
+  const int32_t* cu_seqlens_k;
 } mala_bwd_args;
 
 MALA_API size_t mala_bwd_workspace_size(const mala_bwd_args* args);

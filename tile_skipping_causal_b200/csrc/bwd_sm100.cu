@@ -88,13 +88,26 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // work item: (b, hk, j), smaller j (more query blocks) first
+  // work item: (b, hk, j), smaller j (more query blocks) first; b is the
+  // batch index, or the sequence of a packed call (qrow0 / krow0 its first
+  // query / key row, tb its batch coordinate in the tensor maps)
   const int BK = p.B * p.Hkv;
   const int j = static_cast<int>(blockIdx.x) / BK;
   const int bk = static_cast<int>(blockIdx.x) % BK;
   const int b = bk / p.Hkv;
   const int hk = bk % p.Hkv;
   const int G = p.group_size[hk];
+  int Nq = p.N, Nk = p.Nk, qrow0 = 0, krow0 = 0, tb = b;
+  if (p.seq.n != 0) {
+    qrow0 = p.seq.q0[b];
+    krow0 = p.seq.k0[b];
+    Nq = p.seq.q0[b + 1] - qrow0;
+    Nk = p.seq.k0[b + 1] - krow0;
+    tb = 0;
+    if (j * kB >= Nk) return;       // a shorter sequence: no key block j (uniform exit)
+  }
+  const int q_off = Nk - Nq;        // query q sits at position q + q_off
+  const int nQBs = (Nq + kB - 1) / kB;
 
   if (tid == 0) {
     for (int x = 0; x < kNumBars; ++x) {
@@ -125,21 +138,21 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       tma_prefetch_desc(&p.tm_do);
       mbar_expect_tx(&bars[kKVFull], 2 * kTile);
       for (int c = 0; c < 2; ++c) {
-        tma_load_4d(sK + c * kChunk, &p.tm_k, &bars[kKVFull], c * 64, hk, j * kB, b);
-        tma_load_4d(sV + c * kChunk, &p.tm_v, &bars[kKVFull], c * 64, hk, j * kB, b);
+        tma_load_4d(sK + c * kChunk, &p.tm_k, &bars[kKVFull], c * 64, hk, krow0 + j * kB, tb);
+        tma_load_4d(sV + c * kChunk, &p.tm_v, &bars[kKVFull], c * 64, hk, krow0 + j * kB, tb);
       }
       // scan state of the next visited tile (group head g, query block i);
       // the first query block with a row at or after key block j's first key
       // (query q sits at position q + q_off)
-      const int i_first = max(0, j * kB - p.q_off) / kB;
+      const int i_first = max(0, j * kB - q_off) / kB;
       int sg = 0, si = i_first;
       auto next_tile = [&](int& h_out, int& i_out) -> bool {
         while (sg < G) {
           const int h = p.group_heads[hk][sg];
-          const int64_t bh = static_cast<int64_t>(b) * p.Hq + h;
-          while (si < p.nQB) {
+          while (si < nQBs) {
             const int i = si++;
-            if (!p.fwd_mask || ((p.fwd_mask[(bh * p.nQB + i) * p.mask_words + (j >> 5)] >> (j & 31)) & 1u)) {
+            if (!p.fwd_mask ||
+                ((p.fwd_mask[qblock_index(p.seq, p.Hq, p.nQB, b, h, i) * p.mask_words + (j >> 5)] >> (j & 31)) & 1u)) {
               h_out = h;
               i_out = i;
               return true;
@@ -169,8 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         misc[8 + st] = static_cast<uint32_t>(i);
         mbar_expect_tx(&bars[kQFull + st], kTile + 3 * 512);
         for (int c = 0; c < 2; ++c)
-          tma_load_4d(sQ + st * kTile + c * kChunk, &p.tm_q, &bars[kQFull + st], c * 64, h, i * kB, b);
-        const int64_t row0 = (static_cast<int64_t>(b) * p.Hq + h) * p.Npad + static_cast<int64_t>(i) * kB;
+          tma_load_4d(sQ + st * kTile + c * kChunk, &p.tm_q, &bars[kQFull + st], c * 64, h, qrow0 + i * kB, tb);
+        const int64_t row0 = qblock_index(p.seq, p.Hq, p.nQB, b, h, i) * kB;
         float* sst = sStats + st * 384;
         bulk_load(sst, p.zl2 + row0, 512, &bars[kQFull + st]);
         bulk_load(sst + 128, p.t2 + row0, 512, &bars[kQFull + st]);
@@ -196,7 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
           if (!ok) break;
           mbar_expect_tx(&bars[kDoFull], kTile);
           for (int c = 0; c < 2; ++c)
-            tma_load_4d(sDO + c * kChunk, &p.tm_do, &bars[kDoFull], c * 64, info_h[n & 3], info_i[n & 3] * kB, b);
+            tma_load_4d(sDO + c * kChunk, &p.tm_do, &bars[kDoFull], c * 64, info_h[n & 3],
+                        qrow0 + info_i[n & 3] * kB, tb);
           ++kc_load;
         }
         if (n_total < 0) {
@@ -338,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       reg_fence(q1);
       tc_fence_before();
       mbar_arrive(&bars[kYFree]);
-      float* dst = p.dq_acc + ((static_cast<int64_t>(b) * p.Hq + pend_h) * p.nQB + pend_i) * (kB * kD) + r * 4;
+      float* dst = p.dq_acc + qblock_index(p.seq, p.Hq, p.nQB, b, pend_h, pend_i) * (kB * kD) + r * 4;
 #pragma unroll
       for (int u = 0; u < 8; ++u)
         red_add_v4_f32(dst + (c0 / 4 + u) * (kB * 4), __uint_as_float(q0[4 * u]), __uint_as_float(q0[4 * u + 1]),
@@ -367,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       const bool oks = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], n & 1, abort_flag, p.err, wait_tag(0, kSFull, n)));
       // first legal column of this half for key row r: query column c is at
       // position i * 128 + c + q_off and sees key j * 128 + r iff that is >= it
-      const int lim = (j * kB + r) - (i * kB + p.q_off) - c0;
+      const int lim = (j * kB + r) - (i * kB + q_off) - c0;
       uint32_t sr[2][32];
       if (oks) {
         tc_fence_after();
@@ -401,9 +415,9 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         ++visited;
         if (keep) {
           ++kept;
-          slots += static_cast<int64_t>(kB) * min(kB, p.N - i * kB);
+          slots += static_cast<int64_t>(kB) * min(kB, Nq - i * kB);
           if (p.bwd_mask)
-            atomicOr(&p.bwd_mask[((static_cast<int64_t>(b) * p.Hq + h) * p.nQB + i) * p.mask_words + (j >> 5)],
+            atomicOr(&p.bwd_mask[qblock_index(p.seq, p.Hq, p.nQB, b, h, i) * p.mask_words + (j >> 5)],
                      1u << (j & 31));
         }
       }
@@ -496,8 +510,10 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
     if (okdone && !*abort_flag) {
       tc_fence_after();
       const bool any_kept = kc > 0;            // dK/dV TMEM untouched when nothing was retained
-      __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(p.dk) + b * p.dk_sb + static_cast<int64_t>(krow) * p.dk_sn + hk * p.dk_sh;
-      __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(p.dv) + b * p.dv_sb + static_cast<int64_t>(krow) * p.dv_sn + hk * p.dv_sh;
+      __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(p.dk) + tb * p.dk_sb +
+                           static_cast<int64_t>(krow0 + krow) * p.dk_sn + hk * p.dk_sh;
+      __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(p.dv) + tb * p.dv_sb +
+                           static_cast<int64_t>(krow0 + krow) * p.dv_sn + hk * p.dv_sh;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t base = which == 0 ? tDK : tDV;
@@ -508,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
           tmem_ld32(base + lane_addr + c0 + c * 32, rr);
           tmem_ld_wait(rr);
           reg_fence(rr);
-          if (krow < p.Nk) {
+          if (krow < Nk) {
             uint32_t pk[16];
 #pragma unroll
             for (int x = 0; x < 32; x += 2)
@@ -538,19 +554,56 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
 // D = rowsum(dO o O), zl2 = z log2e, t2 = z + log tau - log(q + 1) (the
 // score a legal entry must reach to retain the tile, natural log units),
 // padded rows: zl2 = t2 = +inf, D = 0; zero the block's dQ accumulator.
+// Query block of an auxiliary CTA: blk = qblock_index(b, h, i); the
+// sequence's first query row, batch coordinate, length and offset.
+struct AuxBlock {
+  int b, h, i, qrow0, tb, Nq, q_off;
+};
+
+__device__ __forceinline__ AuxBlock aux_block(const BwdAuxParams& p, int blk) {
+  AuxBlock a;
+  if (p.seq.n == 0) {
+    a.i = blk % p.nQB;
+    const int bh = blk / p.nQB;
+    a.b = bh / p.Hq;
+    a.h = bh % p.Hq;
+    a.qrow0 = 0;
+    a.tb = a.b;
+    a.Nq = p.N;
+    a.q_off = p.q_off;
+  } else {
+    const int QB = p.seq.qb0[p.seq.n];
+    a.h = blk / QB;
+    const int gqb = blk % QB;
+    int lo = 0, hi = p.seq.n - 1;             // the sequence with qb0[s] <= gqb < qb0[s + 1]
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.seq.qb0[mid] <= gqb) lo = mid; else hi = mid - 1;
+    }
+    while (p.seq.qb0[lo + 1] <= gqb) ++lo;      // skip sequences without query blocks
+    a.b = lo;
+    a.i = gqb - p.seq.qb0[lo];
+    a.qrow0 = p.seq.q0[lo];
+    a.tb = 0;
+    a.Nq = p.seq.q0[lo + 1] - a.qrow0;
+    a.q_off = (p.seq.k0[lo + 1] - p.seq.k0[lo]) - a.Nq;
+  }
+  return a;
+}
+
 __global__ void __launch_bounds__(128) mala_bwd_pre_kernel(const __grid_constant__ BwdAuxParams p) {
-  const int blk = blockIdx.x;                  // (b, h, i)
-  const int i = blk % p.nQB;
-  const int bh = blk / p.nQB;
-  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int blk = blockIdx.x;                  // qblock_index(b, h, i)
+  const AuxBlock ab = aux_block(p, blk);
+  const int b = ab.tb, h = ab.h, i = ab.i;
   const int t = threadIdx.x;
   const int q = i * kB + t;
-  const int64_t row = static_cast<int64_t>(bh) * p.Npad + q;
-  if (q < p.N) {
+  const int64_t row = static_cast<int64_t>(blk) * kB + t;
+  if (q < ab.Nq) {
+    const int64_t qr = ab.qrow0 + q;
     const uint4* o4 = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.o) + b * p.o_sb +
-                                                     static_cast<int64_t>(q) * p.o_sn + h * p.o_sh);
+                                                     qr * p.o_sn + h * p.o_sh);
     const uint4* g4 = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.dout) + b * p.do_sb +
-                                                     static_cast<int64_t>(q) * p.do_sn + h * p.do_sh);
+                                                     qr * p.do_sn + h * p.do_sh);
     float acc = 0.0f;
 #pragma unroll
     for (int u = 0; u < kD / 8; ++u) {
@@ -565,31 +618,32 @@ __global__ void __launch_bounds__(128) mala_bwd_pre_kernel(const __grid_constant
         acc = fmaf(af.y, gf.y, acc);
       }
     }
-    const float z = p.lse[static_cast<int64_t>(bh) * p.N + q];
+    // lse: [B, H_q, N_q], or [H_q, total_q] for packed sequences
+    const float z = p.seq.n == 0 ? p.lse[(static_cast<int64_t>(ab.b) * p.Hq + h) * p.N + q]
+                                 : p.lse[static_cast<int64_t>(h) * p.seq.q0[p.seq.n] + qr];
     p.Dv[row] = acc;
     p.zl2[row] = z * kLog2e;
-    p.t2[row] = z + p.log_tau - logf(static_cast<float>(q + p.q_off + 1));
+    p.t2[row] = z + p.log_tau - logf(static_cast<float>(q + ab.q_off + 1));
   } else {
     p.Dv[row] = 0.0f;
     p.zl2[row] = INFINITY;
     p.t2[row] = INFINITY;
   }
-  float4* acc4 = reinterpret_cast<float4*>(p.dq_acc + (static_cast<int64_t>(bh) * p.nQB + i) * (kB * kD));
+  float4* acc4 = reinterpret_cast<float4*>(p.dq_acc + static_cast<int64_t>(blk) * (kB * kD));
   for (int e = t; e < kB * kD / 4; e += 128) acc4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // dQ (bf16, [B, N, Hq, d]) from the blocked fp32 accumulator
 // [B, Hq, nQB, 32 column quads, 128 rows, 4].
 __global__ void __launch_bounds__(128) mala_bwd_dq_kernel(const __grid_constant__ BwdAuxParams p) {
-  const int blk = blockIdx.x;
-  const int i = blk % p.nQB;
-  const int bh = blk / p.nQB;
-  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int blk = blockIdx.x;                  // qblock_index(b, h, i)
+  const AuxBlock ab = aux_block(p, blk);
   const int t = threadIdx.x;
-  const int q = i * kB + t;
-  if (q >= p.N) return;
-  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + (static_cast<int64_t>(bh) * p.nQB + i) * (kB * kD)) + t;
-  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.dq) + b * p.dq_sb + static_cast<int64_t>(q) * p.dq_sn + h * p.dq_sh;
+  const int q = ab.i * kB + t;
+  if (q >= ab.Nq) return;
+  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + static_cast<int64_t>(blk) * (kB * kD)) + t;
+  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.dq) + ab.tb * p.dq_sb +
+                       static_cast<int64_t>(ab.qrow0 + q) * p.dq_sn + ab.h * p.dq_sh;
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
   for (int u = 0; u < 16; ++u) {
@@ -605,7 +659,8 @@ __global__ void __launch_bounds__(128) mala_bwd_dq_kernel(const __grid_constant_
 size_t bwd_smem_bytes() { return Smem::kAlloc; }
 
 cudaError_t launch_bwd(const BwdParams& p, const BwdAuxParams& aux, cudaStream_t stream) {
-  const unsigned blocks_q = static_cast<unsigned>(aux.B) * aux.Hq * aux.nQB;
+  const unsigned blocks_q = aux.seq.n == 0 ? static_cast<unsigned>(aux.B) * aux.Hq * aux.nQB
+                                           : static_cast<unsigned>(aux.Hq) * aux.seq.qb0[aux.seq.n];
   mala_bwd_pre_kernel<<<blocks_q, 128, 0, stream>>>(aux);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -122,17 +122,38 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // ---- work item: query blocks with more key tiles first
-  const int BH = p.B * p.Hq;
-  const int i = p.nQB - 1 - static_cast<int>(blockIdx.x) / BH;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
-  const int b = bh / p.Hq;
-  const int h = bh % p.Hq;
+  // ---- work item: query blocks with more key tiles first. b is the batch
+  // index, or the sequence of a packed call; qrow0 / krow0 are the sequence's
+  // first query / key row and tb its batch coordinate in the tensor maps.
+  int i, b, h, Nq, Nk, qrow0, krow0, tb;
+  if (p.seq.n == 0) {
+    const int BH = p.B * p.Hq;
+    i = p.nQB - 1 - static_cast<int>(blockIdx.x) / BH;
+    const int bh = static_cast<int>(blockIdx.x) % BH;
+    b = bh / p.Hq;
+    h = bh % p.Hq;
+    Nq = p.N;
+    Nk = p.Nk;
+    qrow0 = krow0 = 0;
+    tb = b;
+  } else {
+    const int SH = p.seq.n * p.Hq;
+    i = p.nQB - 1 - static_cast<int>(blockIdx.x) / SH;
+    const int sh = static_cast<int>(blockIdx.x) % SH;
+    b = sh / p.Hq;
+    h = sh % p.Hq;
+    qrow0 = p.seq.q0[b];
+    krow0 = p.seq.k0[b];
+    Nq = p.seq.q0[b + 1] - qrow0;
+    Nk = p.seq.k0[b + 1] - krow0;
+    tb = 0;
+    if (i * kBQ >= Nq) return;      // a shorter sequence: no query block i (uniform exit)
+  }
+  const int q_off = Nk - Nq;        // bottom-right alignment: query row q sits at position q + q_off
   const int hk = p.kv_of_q[h];
   const int q0 = i * kBQ;
-  const int last_row = min(q0 + kBQ - 1, p.N - 1);
-  // bottom-right alignment: query row q sits at position q + q_off
-  const int j_diag = min((last_row + p.q_off) / kBK, p.nKB - 1);
+  const int last_row = min(q0 + kBQ - 1, Nq - 1);
+  const int j_diag = min((last_row + q_off) / kBK, (Nk + kBK - 1) / kBK - 1);
   const int T = j_diag + 1;         // tile t visits key block j = j_diag - t
 
   if (tid == 0) {
@@ -163,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       tma_prefetch_desc(&p.tm_v);
       mbar_expect_tx(&bars[kQFull], L::kTile);
       for (int c = 0; c < NCH; ++c)
-        tma_load_4d(sQ + c * kChunkBytes, &p.tm_q, &bars[kQFull], c * 64, h, q0, b);
+        tma_load_4d(sQ + c * kChunkBytes, &p.tm_q, &bars[kQFull], c * 64, h, qrow0 + q0, tb);
       misc[2] = 0x10000u;
       int next_k = 0, next_d = 0, v_issued = 0, v_req = 0;
       int vq[8];                         // retained tiles waiting for their V load
@@ -177,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
             mbar_expect_tx(&bars[kKFull + s], L::kTile);
             for (int c = 0; c < NCH; ++c)
               tma_load_4d(sK + s * L::kTile + c * kChunkBytes, &p.tm_k, &bars[kKFull + s], c * 64, hk,
-                          (j_diag - next_k) * kBK, b);
+                          krow0 + (j_diag - next_k) * kBK, tb);
             ++next_k;
             progress = true;
           }
@@ -199,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
             mbar_expect_tx(&bars[kVFull + s], L::kTile);
             for (int c = 0; c < NCH; ++c)
               tma_load_4d(sV + s * L::kTile + c * kChunkBytes, &p.tm_v, &bars[kVFull + s], c * 64, hk,
-                          (j_diag - t) * kBK, b);
+                          krow0 + (j_diag - t) * kBK, tb);
             ++v_issued;
             progress = true;
           }
@@ -287,8 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
     const int g = warp >> 2;                    // column group: key columns [64g, 64g + 64)
     const int c0 = g * 64;
     const int q = q0 + r;
-    const bool valid = q < p.N;
-    const int qa = q + p.q_off;                 // the row's position: keys k <= qa are legal
+    const bool valid = q < Nq;
+    const int qa = q + q_off;                   // the row's position: keys k <= qa are legal
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float thr2 = p.log2_tau - log2f(static_cast<float>(qa + 1));   // log2(tau / L_q)
     float m2 = -INFINITY;                    // reference maximum, log2 units
@@ -297,7 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
     bool prev_kept = false;
     uint32_t mask_word = 0;
     int kept_tiles = 0;
-    const int mask_base = ((b * p.Hq + h) * p.nQB + i) * p.mask_words;
+    const int mask_base = (p.seq.n == 0 ? (b * p.Hq + h) * p.nQB + i
+                                        : h * p.seq.qb0[p.seq.n] + p.seq.qb0[b] + i) * p.mask_words;
     if (tid == 0 && p.keep_mask) {
       for (int w = j_diag / 32 + 1; w < p.mask_words; ++w) p.keep_mask[mask_base + w] = 0u;
     }
@@ -326,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       // block's first row position can hold illegal keys (the diagonal
       // tile, and the one before it when q_off is not a multiple of 128).
       const bool has_key = valid && qa >= j * kBK;
-      if (j * kBK + kBK - 1 > q0 + p.q_off) {
+      if (j * kBK + kBK - 1 > q0 + q_off) {
         const int lim = qa - j * kBK - c0;    // largest legal x
 #pragma unroll
         for (int x = 0; x < 64; ++x)
@@ -444,8 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
                   wait_tag(0, kTileDone + (T - 1) % kNS, T - 1));
       tc_fence_after();
       const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + b * p.o_sb +
-                            static_cast<int64_t>(q) * p.o_sn + h * p.o_sh;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + static_cast<int64_t>(tb) * p.o_sb +
+                            static_cast<int64_t>(qrow0 + q) * p.o_sn + h * p.o_sh;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t o[32];
@@ -463,7 +485,12 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
           for (int u = 0; u < 4; ++u) dst[u] = make_uint4(pko[4 * u], pko[4 * u + 1], pko[4 * u + 2], pko[4 * u + 3]);
         }
       }
-      if (valid && g == 0) p.lse[(static_cast<int64_t>(b) * p.Hq + h) * p.N + q] = (m2 + log2f(l)) * kLn2;
+      if (valid && g == 0) {
+        // [B, H_q, N_q], or [H_q, total_q] for packed sequences
+        const int64_t li = p.seq.n == 0 ? (static_cast<int64_t>(b) * p.Hq + h) * p.N + q
+                                        : static_cast<int64_t>(h) * p.seq.q0[p.seq.n] + qrow0 + q;
+        p.lse[li] = (m2 + log2f(l)) * kLn2;
+      }
       if (tid == 0 && p.stats) {
         const int nvalid = last_row - q0 + 1;
         atomicAdd(reinterpret_cast<unsigned long long*>(&p.stats[0]), static_cast<unsigned long long>(T));

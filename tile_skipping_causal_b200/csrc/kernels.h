@@ -11,6 +11,18 @@ namespace mala {
 constexpr int kMaxHeads = 256;
 
 // Forward, tensor-core path (bf16, B_q = B_k = 128).
+// Packed variable-length sequences (n = 0: fixed lengths, batch dimension
+// used instead). Sequence s owns query rows [q0[s], q0[s+1]) and key rows
+// [k0[s], k0[s+1]) of the packed tensors; its query blocks are numbered from
+// qb0[s] in the packed mask and workspace layouts.
+constexpr int kMaxSeqs = 128;
+struct SeqTable {
+  int n;
+  int q0[kMaxSeqs + 1];
+  int k0[kMaxSeqs + 1];
+  int qb0[kMaxSeqs + 1];
+};
+
 struct FwdTcParams {
   CUtensorMap tm_q;     // [B, N, Hq, D] as 4-D {D, Hq, N, B}, box {64, 1, 128, 1}, 128B swizzle
   CUtensorMap tm_k;     // [B, N, Hkv, D]
@@ -26,6 +38,7 @@ struct FwdTcParams {
   int nQB, nKB, mask_words;
   float log2_tau;       // log2(tau): -inf for tau = 0, +inf for tau = inf
   uint8_t kv_of_q[kMaxHeads];
+  SeqTable seq;         // packed sequences: nQB / nKB / mask_words are then maxima
 };
 
 cudaError_t launch_fwd_tc(const FwdTcParams& p, int head_dim, cudaStream_t stream);
@@ -95,6 +108,7 @@ struct BwdParams {
   int Nk, q_off;           // N_k >= N_q; query q sits at position q + q_off
   uint8_t group_size[kMaxKvHeads];
   uint8_t group_heads[kMaxKvHeads][kMaxGroup];
+  SeqTable seq;            // packed sequences (B = their number; nQB / nKB maxima)
 };
 
 struct BwdAuxParams {      // pre-pass and dQ conversion
@@ -110,7 +124,17 @@ struct BwdAuxParams {      // pre-pass and dQ conversion
   int B, Hq, N, Npad, nQB;   // N = N_q
   int q_off;                 // query q sits at position q + q_off: L_q = q + q_off + 1
   float log_tau;
+  SeqTable seq;              // packed sequences (B = their number)
 };
+
+// Index of query block i of (batch or packed sequence b, query head h) in
+// the [.., 128 rows] workspace blocks, the dQ accumulator and the mask rows:
+// (b H_q + h) nQB + i for fixed lengths, h QB + qb0[b] + i for packed
+// sequences (QB = all packed query blocks).
+__host__ __device__ inline int64_t qblock_index(const SeqTable& seq, int Hq, int nQB, int b, int h, int i) {
+  return seq.n == 0 ? (static_cast<int64_t>(b) * Hq + h) * nQB + i
+                    : static_cast<int64_t>(h) * seq.qb0[seq.n] + seq.qb0[b] + i;
+}
 
 cudaError_t launch_bwd(const BwdParams& p, const BwdAuxParams& aux, cudaStream_t stream);
 size_t bwd_smem_bytes();

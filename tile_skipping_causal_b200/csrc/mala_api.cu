@@ -8,10 +8,13 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "kernels.h"
 #include "mala.h"
+
+static_assert(MALA_MAX_SEQS == mala::kMaxSeqs, "packed-sequence limit of the header and the kernels differ");
 
 namespace mala {
 // {code, tag, block, parity, progress x3, spare} of the first device-side
@@ -164,6 +167,37 @@ int mala_check_device_error(void* stream) {
   return MALA_OK;
 }
 
+// Packed variable-length sequences: checks the host offset arrays and fills
+// the kernels' sequence table; nQB / nKB receive the per-sequence maxima.
+int seq_table(const int32_t* cq, const int32_t* ck, int64_t nseq, int64_t total_q, int64_t total_k,
+              mala::SeqTable* t, int* nQB, int* nKB) {
+  if (!cq || !ck) return fail(MALA_ERR_INVALID_ARG, "packed sequences need both cu_seqlens_q and cu_seqlens_k");
+  if (nseq > mala::kMaxSeqs) return fail(MALA_ERR_UNSUPPORTED, "more than %d packed sequences", mala::kMaxSeqs);
+  if (cq[0] != 0 || ck[0] != 0) return fail(MALA_ERR_INVALID_ARG, "cu_seqlens must start at 0");
+  if (cq[nseq] != total_q || ck[nseq] != total_k)
+    return fail(MALA_ERR_INVALID_ARG, "cu_seqlens must end at seqlen_q / seqlen_k (the packed totals)");
+  t->n = static_cast<int>(nseq);
+  *nQB = *nKB = 1;
+  int qb = 0;
+  for (int64_t s = 0; s < nseq; ++s) {
+    const int64_t lq = static_cast<int64_t>(cq[s + 1]) - cq[s], lk = static_cast<int64_t>(ck[s + 1]) - ck[s];
+    if (lq < 0 || lk < 0) return fail(MALA_ERR_INVALID_ARG, "cu_seqlens must be non-decreasing");
+    if (lq > lk)
+      return fail(MALA_ERR_UNSUPPORTED, "sequence %lld has more queries than keys (needs N_q <= N_k)", (long long)s);
+    t->q0[s] = cq[s];
+    t->k0[s] = ck[s];
+    t->qb0[s] = qb;
+    const int bq = static_cast<int>((lq + 127) / 128), bk = static_cast<int>((lk + 127) / 128);
+    qb += bq;
+    *nQB = std::max(*nQB, bq);
+    *nKB = std::max(*nKB, bk);
+  }
+  t->q0[nseq] = static_cast<int>(total_q);
+  t->k0[nseq] = static_cast<int>(total_k);
+  t->qb0[nseq] = qb;
+  return MALA_OK;
+}
+
 // ------------------------------------------------------------------ forward
 
 size_t mala_fwd_workspace_size(const mala_fwd_args* a) {
@@ -198,8 +232,16 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
     return fail(MALA_ERR_INVALID_ARG, "stats misaligned");
   const int64_t N = a->seqlen_q;
   const int64_t Nk = a->seqlen_k;
-  const int nQB = static_cast<int>((N + a->block_q - 1) / a->block_q);
-  const int nKB = static_cast<int>((Nk + a->block_k - 1) / a->block_k);
+  int nQB = static_cast<int>((N + a->block_q - 1) / a->block_q);
+  int nKB = static_cast<int>((Nk + a->block_k - 1) / a->block_k);
+  const bool packed = a->cu_seqlens_q || a->cu_seqlens_k;
+  mala::SeqTable seq;
+  seq.n = 0;
+  if (packed) {
+    if (!(a->dtype == MALA_BF16 && a->block_q == 128 && a->block_k == 128))
+      return fail(MALA_ERR_UNSUPPORTED, "packed sequences need bf16 and 128 x 128 tiles");
+    if ((rc = seq_table(a->cu_seqlens_q, a->cu_seqlens_k, a->batch, N, Nk, &seq, &nQB, &nKB))) return rc;
+  }
   const int mask_words = (nKB + 31) / 32;
   if ((double)a->batch * a->heads_q * nQB > 2147483647.0) return fail(MALA_ERR_UNSUPPORTED, "grid too large");
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
@@ -209,9 +251,12 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
     mala::FwdTcParams p;
     memset(&p, 0, sizeof(p));
     if ((rc = head_map(a->q_to_kv, a->heads_q, a->heads_kv, p.kv_of_q))) return rc;
-    if ((rc = make_map_bf16(&p.tm_q, a->q, a->batch, N, a->heads_q, d, a->q_stride, 128))) return rc;
-    if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, Nk, a->heads_kv, d, a->k_stride, 128))) return rc;
-    if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, Nk, a->heads_kv, d, a->v_stride, 128))) return rc;
+    // packed sequences: one batch entry of total_q / total_k rows
+    const int64_t mb = packed ? 1 : a->batch;
+    if ((rc = make_map_bf16(&p.tm_q, a->q, mb, N, a->heads_q, d, a->q_stride, 128))) return rc;
+    if ((rc = make_map_bf16(&p.tm_k, a->k, mb, Nk, a->heads_kv, d, a->k_stride, 128))) return rc;
+    if ((rc = make_map_bf16(&p.tm_v, a->v, mb, Nk, a->heads_kv, d, a->v_stride, 128))) return rc;
+    p.seq = seq;
     p.err = device_error_ptr();
     if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
     p.o = a->o;
@@ -282,6 +327,12 @@ int bwd_check(const mala_bwd_args* a) {
   if (a->seqlen_k > (1 << 30)) return fail(MALA_ERR_UNSUPPORTED, "sequence too long");
   if (a->heads_kv > mala::kMaxKvHeads) return fail(MALA_ERR_UNSUPPORTED, "heads_kv > %d", mala::kMaxKvHeads);
   if (!a->lse) return fail(MALA_ERR_INVALID_ARG, "lse is NULL");
+  if (a->cu_seqlens_q || a->cu_seqlens_k) {
+    mala::SeqTable t;
+    int nQB = 0, nKB = 0;
+    if ((rc = seq_table(a->cu_seqlens_q, a->cu_seqlens_k, a->batch, a->seqlen_q, a->seqlen_k, &t, &nQB, &nKB)))
+      return rc;
+  }
   if ((rc = check_tensor("q", a->q, a->q_stride, 2, 128, a->heads_q))) return rc;
   if ((rc = check_tensor("k", a->k, a->k_stride, 2, 128, a->heads_kv))) return rc;
   if ((rc = check_tensor("v", a->v, a->v_stride, 2, 128, a->heads_kv))) return rc;
@@ -293,10 +344,21 @@ int bwd_check(const mala_bwd_args* a) {
   return MALA_OK;
 }
 
-// workspace: zl2, t2, D ([B, Hq, Npad] fp32 each) then the blocked dQ accumulator
-size_t bwd_ws_bytes(const mala_bwd_args* a) {
+// Rows of the backward workspace: B H_q nQB 128 for fixed lengths, or
+// H_q QB 128 for packed sequences (QB = all packed query blocks).
+size_t bwd_rows(const mala_bwd_args* a) {
+  if (a->cu_seqlens_q) {
+    size_t qb = 0;
+    for (int64_t s = 0; s < a->batch; ++s) qb += static_cast<size_t>((a->cu_seqlens_q[s + 1] - a->cu_seqlens_q[s] + 127) / 128);
+    return static_cast<size_t>(a->heads_q) * qb * 128;
+  }
   const size_t npad = static_cast<size_t>((a->seqlen_q + 127) / 128) * 128;
-  const size_t rows = static_cast<size_t>(a->batch) * a->heads_q * npad;
+  return static_cast<size_t>(a->batch) * a->heads_q * npad;
+}
+
+// workspace: zl2, t2, D (one fp32 per row each) then the blocked dQ accumulator
+size_t bwd_ws_bytes(const mala_bwd_args* a) {
+  const size_t rows = bwd_rows(a);
   return rows * 3 * sizeof(float) + rows * 128 * sizeof(float) + 256;
 }
 
@@ -317,13 +379,15 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
   if (!aligned16(workspace)) return fail(MALA_ERR_INVALID_ARG, "workspace misaligned");
   const int N = static_cast<int>(a->seqlen_q);
   const int Nk = static_cast<int>(a->seqlen_k);
-  const int nQB = (N + 127) / 128;
-  const int nKB = (Nk + 127) / 128;
+  int nQB = (N + 127) / 128;
+  int nKB = (Nk + 127) / 128;
   const int Npad = nQB * 128;
-  const size_t rows = static_cast<size_t>(a->batch) * a->heads_q * Npad;
+  const size_t rows = bwd_rows(a);
+  const bool packed = a->cu_seqlens_q != nullptr;
 
   mala::BwdParams p;
   memset(&p, 0, sizeof(p));
+  if (packed && (rc = seq_table(a->cu_seqlens_q, a->cu_seqlens_k, a->batch, N, Nk, &p.seq, &nQB, &nKB))) return rc;
   uint8_t kv_of_q[mala::kMaxHeads];
   if ((rc = head_map(a->q_to_kv, a->heads_q, a->heads_kv, kv_of_q))) return rc;
   for (int64_t h = 0; h < a->heads_q; ++h) {
@@ -332,10 +396,11 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
       return fail(MALA_ERR_UNSUPPORTED, "more than %d query heads share KV head %d", mala::kMaxGroup, hk);
     p.group_heads[hk][p.group_size[hk]++] = static_cast<uint8_t>(h);
   }
-  if ((rc = make_map_bf16(&p.tm_q, a->q, a->batch, N, a->heads_q, 128, a->q_stride, 128))) return rc;
-  if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, Nk, a->heads_kv, 128, a->k_stride, 128))) return rc;
-  if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, Nk, a->heads_kv, 128, a->v_stride, 128))) return rc;
-  if ((rc = make_map_bf16(&p.tm_do, a->dout, a->batch, N, a->heads_q, 128, a->do_stride, 128))) return rc;
+  const int64_t mb = packed ? 1 : a->batch;   // packed sequences: one batch entry of total rows
+  if ((rc = make_map_bf16(&p.tm_q, a->q, mb, N, a->heads_q, 128, a->q_stride, 128))) return rc;
+  if ((rc = make_map_bf16(&p.tm_k, a->k, mb, Nk, a->heads_kv, 128, a->k_stride, 128))) return rc;
+  if ((rc = make_map_bf16(&p.tm_v, a->v, mb, Nk, a->heads_kv, 128, a->v_stride, 128))) return rc;
+  if ((rc = make_map_bf16(&p.tm_do, a->dout, mb, N, a->heads_q, 128, a->do_stride, 128))) return rc;
   float* ws = static_cast<float*>(workspace);
   p.zl2 = ws;
   p.t2 = ws + rows;
@@ -380,12 +445,14 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
   x.Npad = Npad;
   x.nQB = nQB;
   x.q_off = Nk - N;
+  x.seq = p.seq;
   x.log_tau = a->tau == 0.0f ? -INFINITY : logf(a->tau);
 
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (a->bwd_keep_mask) {
-    cudaError_t e = cudaMemsetAsync(a->bwd_keep_mask, 0,
-                                    static_cast<size_t>(a->batch) * a->heads_q * nQB * p.mask_words * 4, stream);
+    const size_t mrows = packed ? static_cast<size_t>(a->heads_q) * p.seq.qb0[p.seq.n]
+                                : static_cast<size_t>(a->batch) * a->heads_q * nQB;
+    cudaError_t e = cudaMemsetAsync(a->bwd_keep_mask, 0, mrows * p.mask_words * 4, stream);
     if (e != cudaSuccess) return cuda_fail(e, "backward mask clear");
   }
   cudaError_t e = mala::launch_bwd(p, x, stream);

@@ -35,7 +35,7 @@ class FwdArgs(ctypes.Structure):
         ("q_stride", _i64x3), ("k_stride", _i64x3), ("v_stride", _i64x3), ("o_stride", _i64x3),
         ("q_to_kv", ctypes.c_void_p), ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32),
         ("tau", ctypes.c_float), ("dtype", ctypes.c_int32), ("mode", ctypes.c_int32),
-        ("stats", ctypes.c_void_p),
+        ("stats", ctypes.c_void_p), ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
     ]
 
 
@@ -51,6 +51,7 @@ class BwdArgs(ctypes.Structure):
         ("do_stride", _i64x3), ("dq_stride", _i64x3), ("dk_stride", _i64x3), ("dv_stride", _i64x3),
         ("q_to_kv", ctypes.c_void_p), ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32),
         ("tau", ctypes.c_float), ("dtype", ctypes.c_int32), ("stats", ctypes.c_void_p),
+        ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
     ]
 
 
@@ -209,45 +210,85 @@ def fwd_args(q, k, v, o, lse, keep_mask, tau, block_q, block_k, stats=None, q_to
     return a
 
 
+def _packed(cu_seqlens_q, cu_seqlens_k, block_q, block_k):
+    """Host int32 offset arrays of packed sequences -> (arrays, number of
+    sequences, packed query blocks, largest key-block count)."""
+    cq = np.ascontiguousarray(np.asarray(cu_seqlens_q, dtype=np.int32))
+    ck = np.ascontiguousarray(np.asarray(cu_seqlens_k, dtype=np.int32))
+    if cq.shape != ck.shape or cq.ndim != 1 or cq.size < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must be 1-D arrays of equal length >= 2")
+    lq, lk = np.diff(cq.astype(np.int64)), np.diff(ck.astype(np.int64))
+    QB = int((-(-lq // block_q)).sum())
+    KB = max(1, int((-(-lk // block_k)).max()))
+    return cq, ck, cq.size - 1, QB, KB
+
+
 def mala_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float,
              block_q: int = 128, block_k: int = 128, *, o=None, lse=None, keep_mask=None,
-             with_mask: bool = True, stats=None, q_to_kv=None, stream=None):
-    """MALA forward/prefill. q [B, N, Hq, d], k/v [B, N, Hkv, d] (bf16 or fp32,
-    scale folded into q). Returns (o, lse [B, Hq, N] fp32, keep_mask words
-    [B, Hq, nQB, ceil(nKB/32)] int32 or None)."""
+             with_mask: bool = True, stats=None, q_to_kv=None, stream=None,
+             cu_seqlens_q=None, cu_seqlens_k=None):
+    """MALA forward/prefill. q [B, N_q, Hq, d], k/v [B, N_k, Hkv, d] (bf16 or
+    fp32, scale folded into q; N_q <= N_k, bottom-right aligned). Returns
+    (o, lse [B, Hq, N_q] fp32, keep_mask words [B, Hq, nQB, ceil(nKB/32)]
+    int32 or None).
+
+    Packed sequences: cu_seqlens_q / cu_seqlens_k (host int32 offsets, one
+    more than the number of sequences) with q [1, total_q, Hq, d] and k, v
+    [1, total_k, Hkv, d]; lse is then [Hq, total_q] and keep_mask
+    [Hq, packed query blocks, ceil(largest key-block count / 32)]."""
     lib = load_library()
     _require_cuda(q, k, v)
     B, N, Hq, d = q.shape
     nQB, nKB = -(-N // block_q), -(-k.shape[1] // block_k)
+    packed = None
+    if cu_seqlens_q is not None or cu_seqlens_k is not None:
+        if q.shape[0] != 1 or k.shape[0] != 1:
+            raise ValueError("packed sequences take q, k, v with a batch dimension of 1")
+        packed = _packed(cu_seqlens_q, cu_seqlens_k, block_q, block_k)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
-        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+        shape = (Hq, N) if packed else (B, Hq, N)
+        lse = torch.empty(shape, dtype=torch.float32, device=q.device)
     if keep_mask is None and with_mask:
-        keep_mask = torch.empty((B, Hq, nQB, mask_words(nKB)), dtype=torch.int32, device=q.device)
+        shape = (Hq, packed[3], mask_words(packed[4])) if packed else (B, Hq, nQB, mask_words(nKB))
+        keep_mask = torch.empty(shape, dtype=torch.int32, device=q.device)
     keep_alive, hm = _head_map(q_to_kv)
     a = fwd_args(q, k, v, o, lse, keep_mask, tau, block_q, block_k, stats, hm)
+    if packed:
+        a.batch = packed[2]
+        a.cu_seqlens_q = packed[0].ctypes.data
+        a.cu_seqlens_k = packed[1].ctypes.data
     ws_n = lib.mala_fwd_workspace_size(ctypes.byref(a))
     ws = torch.empty(ws_n, dtype=torch.uint8, device=q.device) if ws_n else None
     _check(lib.mala_fwd(ctypes.byref(a), _ptr(ws), ws_n, _stream(stream)))
-    del keep_alive
+    del keep_alive, packed
     return o, lse, keep_mask
 
 
 def mala_bwd(q, k, v, o, do, lse, tau: float, keep_mask=None, block_q: int = 128,
              block_k: int = 128, *, dq=None, dk=None, dv=None, bwd_keep_mask=None,
-             with_bwd_mask: bool = False, stats=None, q_to_kv=None, stream=None):
-    """MALA backward. Returns (dq, dk, dv, bwd_keep_mask or None)."""
+             with_bwd_mask: bool = False, stats=None, q_to_kv=None, stream=None,
+             cu_seqlens_q=None, cu_seqlens_k=None):
+    """MALA backward. Returns (dq, dk, dv, bwd_keep_mask or None). Packed
+    sequences as for mala_fwd (the same cu_seqlens; lse and keep_mask in
+    mala_fwd's packed layouts)."""
     lib = load_library()
     _require_cuda(q, k, v, o, do, lse)
     B, N, Hq, d = q.shape
     _, Nk, Hkv, _ = k.shape
     nQB, nKB = -(-N // block_q), -(-Nk // block_k)
+    packed = None
+    if cu_seqlens_q is not None or cu_seqlens_k is not None:
+        if q.shape[0] != 1 or k.shape[0] != 1:
+            raise ValueError("packed sequences take q, k, v with a batch dimension of 1")
+        packed = _packed(cu_seqlens_q, cu_seqlens_k, block_q, block_k)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     if bwd_keep_mask is None and with_bwd_mask:
-        bwd_keep_mask = torch.empty((B, Hq, nQB, mask_words(nKB)), dtype=torch.int32, device=q.device)
+        shape = (Hq, packed[3], mask_words(packed[4])) if packed else (B, Hq, nQB, mask_words(nKB))
+        bwd_keep_mask = torch.empty(shape, dtype=torch.int32, device=q.device)
     keep_alive, hm = _head_map(q_to_kv)
     a = BwdArgs()
     a.q, a.k, a.v, a.o, a.dout = _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do)
@@ -262,10 +303,16 @@ def mala_bwd(q, k, v, o, do, lse, tau: float, keep_mask=None, block_q: int = 128
     a.tau = float(tau)
     a.dtype = _dtype_code(q)
     a.stats = _ptr(stats)
+    if packed:
+        a.batch = packed[2]
+        a.cu_seqlens_q = packed[0].ctypes.data
+        a.cu_seqlens_k = packed[1].ctypes.data
     ws_n = lib.mala_bwd_workspace_size(ctypes.byref(a))
-    ws = torch.empty(ws_n, dtype=torch.uint8, device=q.device) if ws_n else None
+    if ws_n == 0:
+        _check(lib.mala_bwd(ctypes.byref(a), None, 0, _stream(stream)))   # reports the argument error
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=q.device)
     _check(lib.mala_bwd(ctypes.byref(a), _ptr(ws), ws_n, _stream(stream)))
-    del keep_alive
+    del keep_alive, packed
     return dq, dk, dv, bwd_keep_mask
 
 
