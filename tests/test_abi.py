@@ -139,3 +139,65 @@ def test_mask_pack_roundtrip():
     w = torch.from_numpy(mala.pack_mask(m))
     assert w.shape == (2, 3, 5, 3)
     assert (mala.unpack_mask(w, 70) == m).all()
+
+
+# ------------------------------------------------- packed sequences (host checks)
+
+def _cu(*vals):
+    arr = (ctypes.c_int32 * len(vals))(*vals)
+    return arr, ctypes.cast(arr, ctypes.c_void_p)
+
+
+@pytest.mark.parametrize("cq,ck,extra,code", [
+    ((0, 100, 256), None, {}, mala.MALA_ERR_INVALID_ARG),                  # only one of the two arrays
+    ((1, 100, 256), (0, 100, 256), {}, mala.MALA_ERR_INVALID_ARG),          # not starting at 0
+    ((0, 100, 200), (0, 100, 256), {}, mala.MALA_ERR_INVALID_ARG),          # not ending at the total
+    ((0, -1, 256), (0, 100, 256), {}, mala.MALA_ERR_INVALID_ARG),           # decreasing
+    ((0, 150, 256), (0, 100, 256), {}, mala.MALA_ERR_UNSUPPORTED),          # a sequence with N_q > N_k
+    ((0, 100, 256), (0, 100, 256), {"block_q": 64, "block_k": 64}, mala.MALA_ERR_UNSUPPORTED),
+    ((0, 100, 256), (0, 100, 256), {"dtype": mala.MALA_FP32}, mala.MALA_ERR_UNSUPPORTED),
+])
+def test_packed_offsets_rejected_without_launching(lib, cq, ck, extra, code):
+    keep = []
+    kw = dict(batch=2, **extra)
+    arr, ptr = _cu(*cq)
+    keep.append(arr)
+    kw["cu_seqlens_q"] = ptr
+    if ck is not None:
+        arr, ptr = _cu(*ck)
+        keep.append(arr)
+        kw["cu_seqlens_k"] = ptr
+    a = _fwd_args(**kw)
+    rc = lib.mala_fwd(ctypes.byref(a), None, 0, None)
+    assert rc == code, lib.mala_last_error_message()
+    assert lib.mala_last_error_message().decode()
+
+
+def test_packed_sequence_count_limit(lib):
+    n = 129                                   # one more than the packed-sequence limit
+    cq = [0] + [2 * (s + 1) for s in range(n)]
+    arr_q, ptr_q = _cu(*cq)
+    arr_k, ptr_k = _cu(*cq)
+    a = _fwd_args(batch=n, seqlen_q=cq[-1], seqlen_k=cq[-1], cu_seqlens_q=ptr_q, cu_seqlens_k=ptr_k)
+    assert lib.mala_fwd(ctypes.byref(a), None, 0, None) == mala.MALA_ERR_UNSUPPORTED
+    assert "128" in lib.mala_last_error_message().decode()
+
+
+def test_backward_checks_packed_offsets_too(lib):
+    a = mala.BwdArgs()
+    fake = 0x10000
+    a.q = a.k = a.v = a.o = a.dout = a.lse = a.dq = a.dk = a.dv = fake
+    a.batch, a.heads_q, a.heads_kv = 2, 4, 2
+    a.seqlen_q = a.seqlen_k = 256
+    a.head_dim = 128
+    for s in ("q_stride", "o_stride", "do_stride", "dq_stride"):
+        setattr(a, s, mala._i64x3(256 * 4 * 128, 4 * 128, 128))
+    for s in ("k_stride", "v_stride", "dk_stride", "dv_stride"):
+        setattr(a, s, mala._i64x3(256 * 2 * 128, 2 * 128, 128))
+    a.block_q = a.block_k = 128
+    a.tau = 0.1
+    a.dtype = mala.MALA_BF16
+    arr_q, a.cu_seqlens_q = _cu(0, 200, 256)
+    arr_k, a.cu_seqlens_k = _cu(0, 100, 256)         # the first sequence has more queries than keys
+    assert lib.mala_bwd_workspace_size(ctypes.byref(a)) == 0
+    assert lib.mala_bwd(ctypes.byref(a), None, 0, None) == mala.MALA_ERR_UNSUPPORTED
