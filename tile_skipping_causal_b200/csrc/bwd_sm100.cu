@@ -1,9 +1,10 @@
 // MALA backward (Algorithm 2, "Offline Sparse Probability", and Appendix A.1
 // "Fused backward execution" of the MassAlloc Attention paper) on sm_100a.
 //
-// Key-major: one CTA per (batch, KV head, key block j) accumulates dK_j and
-// dV_j in TMEM over every query head of the group and every query block i
-// ascending from the diagonal whose tile (i, j) the forward retained. For a
+// Key-major: one CTA per (batch or packed sequence, KV head, key block j)
+// accumulates dK_j and dV_j in TMEM over every query head of the group and
+// every query block i ascending from the first one that sees key block j
+// (query q at position q + N_k - N_q) whose tile (i, j) the forward retained. For a
 // visited tile the score tile S^T = K_j Q_i^T is recomputed and tested
 // against the saved log-normaliser: the tile is skipped iff for every legal
 // (q, k) s_qk - z_q < log tau - log L_q. A retained tile loads dO_i and runs

@@ -1,9 +1,11 @@
 // MALA forward (Algorithm 1, "Online Sparse Softmax") on sm_100a tensor cores.
 //
-// One CTA owns one query block I_i of 128 rows of one (batch, query head).
-// Key blocks are visited in descending order from the diagonal (Appendix
-// A.1, "Fused forward execution"); every legal tile is scored, and only a
-// retained tile loads V and runs the online-softmax update and PV.
+// One CTA owns one query block I_i of 128 rows of one (batch, query head),
+// or of one (packed sequence, query head). Query row q sits at position
+// q + N_k - N_q (bottom-right alignment; N_q = N_k for training). Key blocks
+// are visited in descending order from the diagonal (Appendix A.1, "Fused
+// forward execution"); every legal tile is scored, and only a retained tile
+// loads V and runs the online-softmax update and PV.
 //
 // Warp roles (320 threads):
 //   warps 0-7  softmax, two warpgroups: warps 0-3 take key columns [0, 64)
