@@ -76,11 +76,14 @@ int make_map_bf16(CUtensorMap* map, const void* ptr, int64_t B, int64_t N, int64
   return MALA_OK;
 }
 
-// Device address of the error block on the current device.
+// Device address of the error block on the current device (looked up once
+// per device; calls from several host threads are serialised here).
 int* device_error_ptr() {
   static int* ptrs[64] = {nullptr};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (!ptrs[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, mala::g_device_error) != cudaSuccess) return nullptr;
