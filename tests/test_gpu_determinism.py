@@ -58,3 +58,25 @@ def test_decode_is_bitwise_reproducible():
         o, lse, keep, P = mala.mala_decode(qd, k, v, w.tau)
         mala.check_device_error()
         assert torch.equal(o, ref[0]) and torch.equal(lse, ref[1]) and torch.equal(keep, ref[2])
+
+
+def test_caller_stream_gives_the_same_results():
+    """Calls on a caller-given stream (workspaces allocated by the binding
+    are kept alive for that stream) match the calls on the current stream."""
+    w = synth.WORKLOADS["train_8k"]
+    t = {n: x.to(DEV) for n, x in synth.make_prefill(w, 42, batch=1, seqlen=1024).items()}
+    o, lse, keep = mala.mala_fwd(t["q"], t["k"], t["v"], 0.1)
+    dq, dk, dv, _ = mala.mala_bwd(t["q"], t["k"], t["v"], o, t["do"], lse, 0.1, keep)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    o2, lse2, keep2 = mala.mala_fwd(t["q"], t["k"], t["v"], 0.1, stream=side)
+    dq2, dk2, dv2, _ = mala.mala_bwd(t["q"], t["k"], t["v"], o2, t["do"], lse2, 0.1, keep2, stream=side)
+    # allocations on the current stream meanwhile may not reuse the side
+    # stream's workspaces while its kernels run
+    junk = [torch.full((1 << 20,), 7.0, device=DEV) for _ in range(64)]
+    torch.cuda.current_stream().wait_stream(side)
+    mala.check_device_error()
+    del junk
+    assert torch.equal(o, o2) and torch.equal(lse, lse2) and torch.equal(keep, keep2)
+    assert torch.equal(dk, dk2) and torch.equal(dv, dv2)
+    assert (dq.float() - dq2.float()).norm() <= 1e-3 * dq.float().norm()

@@ -165,6 +165,13 @@ def _head_map(q_to_kv: Optional[Sequence[int]]):
     return arr, ctypes.cast(arr, ctypes.c_void_p)
 
 
+def _keep_for_stream(ws: Optional[torch.Tensor], stream) -> None:
+    """A workspace allocated on torch's current stream but used on another
+    must not be handed out again before that stream is done with it."""
+    if ws is not None and stream is not None:
+        ws.record_stream(stream)
+
+
 def _require_cuda(*ts):
     for t in ts:
         if t is not None and not t.is_cuda:
@@ -262,6 +269,7 @@ def mala_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float,
     ws_n = lib.mala_fwd_workspace_size(ctypes.byref(a))
     ws = torch.empty(ws_n, dtype=torch.uint8, device=q.device) if ws_n else None
     _check(lib.mala_fwd(ctypes.byref(a), _ptr(ws), ws_n, _stream(stream)))
+    _keep_for_stream(ws, stream)
     del keep_alive, packed
     return o, lse, keep_mask
 
@@ -312,6 +320,7 @@ def mala_bwd(q, k, v, o, do, lse, tau: float, keep_mask=None, block_q: int = 128
         _check(lib.mala_bwd(ctypes.byref(a), None, 0, _stream(stream)))   # reports the argument error
     ws = torch.empty(ws_n, dtype=torch.uint8, device=q.device)
     _check(lib.mala_bwd(ctypes.byref(a), _ptr(ws), ws_n, _stream(stream)))
+    _keep_for_stream(ws, stream)
     del keep_alive, packed
     return dq, dk, dv, bwd_keep_mask
 
@@ -344,9 +353,12 @@ def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *,
     a.num_splits = int(num_splits)
     a.stats = _ptr(stats)
     ws_n = lib.mala_decode_workspace_size(ctypes.byref(a))
-    if workspace is None or workspace.numel() < ws_n:
+    own_ws = workspace is None or workspace.numel() < ws_n
+    if own_ws:
         workspace = torch.empty(ws_n, dtype=torch.uint8, device=q.device) if ws_n else None
     _check(lib.mala_decode(ctypes.byref(a), _ptr(workspace), ws_n, _stream(stream)))
+    if own_ws:
+        _keep_for_stream(workspace, stream)
     del keep_alive
     return o, lse, keep_mask, int(a.num_splits)
 
