@@ -410,6 +410,7 @@ def bench_chunk(args, q, k, v, stream, peaks, chunk: int = 4096):
     from tile_skipping_causal_b200 import mala
 
     Nk = k.shape[1]
+    chunk = min(chunk, Nk // 2)           # shorter runs (--seqlen) take half of their queries
     qc = q[:, Nk - chunk:]
     stats = torch.zeros(4, dtype=torch.int64, device=q.device)
     o, lse, keep = mala.mala_fwd(qc, k, v, TAU, TILE, TILE, stats=stats)
