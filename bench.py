@@ -342,6 +342,7 @@ def run_mala(args):
     peaks = _peaks()
     chunk = bench_chunk(args, q, k, v, stream, peaks)
     dec = None if args.no_decode else bench_decode(args, dev, stream, peaks)
+    dec8 = None if args.no_decode else bench_decode(args, dev, stream, peaks, e4m3=True)
     kern_f = statistics.mean(fwd_times)
     kern_b = statistics.mean(bwd_times)
     ach_f = fwd_flops / kern_f / 1e12
@@ -392,6 +393,7 @@ def run_mala(args):
     res["chunked_prefill"] = chunk
     if dec is not None:
         res["decode"] = dec
+        res["decode_e4m3"] = dec8
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
     if world > 1:
@@ -435,19 +437,25 @@ def bench_chunk(args, q, k, v, stream, peaks, chunk: int = 4096):
             "tflops_executed": flops / t / 1e12, "frac_of_peak": flops / t / 1e12 / peak}
 
 
-def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072):
+def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072, e4m3: bool = False):
     """Split-KV decode on the largest decode workload (batch 64, 32 query
     heads, 8 KV heads, d = 128, bf16 cache of seqlen_k keys, tau = 0.05).
     The 34 GB cache is drawn on the device with the decode recipe (sink key,
-    16 needles per sequence). HBM roofline on the bytes actually read:
-    every K tile plus the V tiles some head retained, plus the queries and
-    the split partials written and read back."""
+    16 needles per sequence); with e4m3 it is then quantised to e4m3 codes
+    (scale 1, 17 GB). HBM roofline on the bytes actually read: every K tile
+    plus the V tiles some head retained, plus the queries and the split
+    partials written and read back."""
     import torch
     from tile_skipping_causal_b200 import mala, synth
 
     w = synth.decode_workload(args.decode_seqlen or seqlen_k)
     q = synth.make_decode_query(w, SEED).to(dev)
     k, v = synth.fill_decode_cache(w, SEED, q.cpu(), dev, slices=[])
+    if e4m3:
+        k = k.to(torch.float8_e4m3fn)
+        v = v.to(torch.float8_e4m3fn)
+        torch.cuda.empty_cache()
+    esz = k.element_size()
     stats = torch.zeros(4, dtype=torch.int64, device=dev)
     o, lse, keep, P = mala.mala_decode(q, k, v, w.tau, 128, 0, stats=stats)
     mala.check_device_error()
@@ -473,14 +481,15 @@ def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072):
     mala.check_device_error()
     t = e0.elapsed_time(e1) / 1e3 / n
     d = w.head_dim
-    kbytes = w.batch * w.heads_kv * w.seqlen_k * d * 2
-    vbytes = vread * 128 * d * 2
+    kbytes = w.batch * w.heads_kv * w.seqlen_k * d * esz
+    vbytes = vread * 128 * d * esz
     other = w.batch * w.heads_q * d * 2 * 2 + (w.batch * w.heads_q * P * (d + 1) * 4 * 2 if P > 1 else 0)
     total = kbytes + vbytes + other
     gbs = total / t / 1e9
     del k, v
     torch.cuda.empty_cache()
-    return {"workload": w.name, "batch": w.batch, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
+    return {"workload": w.name, "cache": "e4m3" if e4m3 else "bf16", "batch": w.batch, "heads_q": w.heads_q,
+            "heads_kv": w.heads_kv,
             "seqlen_k": w.seqlen_k, "tau": w.tau, "splits": P, "ms": t * 1e3,
             "tokens_per_s": w.batch / t, "tiles_tested": tested, "v_tiles_read": vread,
             "v_read_fraction": vread / tested, "head_tiles_kept_fraction": kept_heads / (tested * w.group),
@@ -488,7 +497,7 @@ def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072):
             "roofline": {"bound": "hbm", "kernel": "mala_decode_split_kernel", "achieved": gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                          "peak_source": f"{peaks['source']} hbm_gbs",
-                         "traffic": NCU_TRAFFIC.get(f"mala_decode_split_kernel@{w.seqlen_k}"),
+                         "traffic": None if e4m3 else NCU_TRAFFIC.get(f"mala_decode_split_kernel@{w.seqlen_k}"),
                          "traffic_note": "ncu DRAM bytes per launch, N_k = 8192 capture scaled by N_k"}}
 
 
@@ -597,6 +606,8 @@ def main():
                     help="decode cache length (default 131072); for profiling captures")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the decode measurement (profiling captures)")
+    ap.add_argument("--decode-e4m3", action="store_true",
+                    help="with --decode-only: an e4m3 cache instead of bf16")
     ap.add_argument("--no-extras", action="store_true",
                     help="time the step only (no tau=0, e2e, baseline); for profiling captures")
     args = ap.parse_args()
@@ -609,7 +620,8 @@ def main():
         mala.load_library()
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
-        print(json.dumps(bench_decode(args, dev, torch.cuda.current_stream(), _peaks())), flush=True)
+        print(json.dumps(bench_decode(args, dev, torch.cuda.current_stream(), _peaks(), e4m3=args.decode_e4m3)),
+              flush=True)
     else:
         run_mala(args)
 

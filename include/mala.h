@@ -63,8 +63,9 @@ enum {
   MALA_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up */
 };
 
-/* element types of Q, K, V, O (and dO, dQ, dK, dV) */
-enum { MALA_BF16 = 0, MALA_FP32 = 1 };
+/* element types of Q, K, V, O (and dO, dQ, dK, dV); MALA_FP8_E4M3 only for
+ * the K / V cache of mala_decode (kv_dtype) */
+enum { MALA_BF16 = 0, MALA_FP32 = 1, MALA_FP8_E4M3 = 2 };
 
 /* masking mode of mala_fwd */
 enum {
@@ -226,6 +227,15 @@ typedef struct {
   int32_t dtype;
   int32_t num_splits;
   int64_t* stats;               /* device int64[4]: tiles tested, V tiles read, head-tiles retained, reserved */
+  /* K / V cache element type: MALA_BF16 (0, the default) or MALA_FP8_E4M3
+   * (OCP e4m3, one byte per element, head_dim 128, strides in elements as
+   * for every tensor). An e4m3 cache holds codes whose values are
+   * code * k_scale for K and code * v_scale for V (positive, finite; unused
+   * for bf16); q stays bf16. The scores then use the query rounded to f16
+   * (exact for |q| >= 2^-14) and P in f16. */
+  int32_t kv_dtype;
+  float k_scale;
+  float v_scale;
 } mala_decode_args;
 
 MALA_API size_t mala_decode_workspace_size(const mala_decode_args* args);

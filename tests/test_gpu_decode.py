@@ -113,3 +113,57 @@ def test_decode_stats():
     assert s[2] == m.sum()                    # head-tiles retained
     grp = m.reshape(1, 8, 4, 16).any(axis=2)  # V read iff some head of the group retains
     assert s[1] == grp.sum()
+
+
+# ------------------------------------------------------------ e4m3 KV cache
+# The decode recipe's cache quantised to OCP e4m3 codes with a scale per
+# tensor; the oracle runs on the dequantised values (code * scale), which
+# are exactly what the kernel computes with.
+
+def _quantise(x, scale):
+    codes = (x.float() / scale).to(torch.float8_e4m3fn)
+    return codes, codes.float() * scale
+
+
+@pytest.mark.parametrize("Nk,splits,scales", [(1000, 1, (1.0, 1.0)), (1000, 3, (0.5, 2.0)),
+                                               (4096, 0, (0.25, 0.75)), (129, 0, (1.0, 0.5))])
+def test_decode_e4m3_cache(Nk, splits, scales):
+    w, q, k, v = _small(2, Nk, seed=7)
+    sk, sv = scales
+    kc, kd = _quantise(k, sk)
+    vc, vd = _quantise(v, sv)
+    stats = torch.zeros(4, dtype=torch.int64, device=DEV)
+    o, lse, keep, P = _decode(q, kc, vc, w.tau, splits, k_scale=sk, v_scale=sv, stats=stats)
+    if splits:
+        assert P == splits
+    rep = check_decode(q, kd, vd, o, lse, keep, w.tau, P)
+    assert rep.heads == 2 * 32
+    assert stats[0].item() == 2 * 8 * -(-Nk // 128)
+
+
+def test_decode_e4m3_large_cache_sampled():
+    """Batch 64, 32 query heads, 8 KV heads, N_k = 16384 (1 GB of e4m3 codes
+    per cache), sampled heads against the oracle."""
+    w = synth.decode_workload(16384)
+    q = synth.make_decode_query(w, SEED)
+    sample_kv = [(0, 0), (40, 5)]
+    k, v = synth.fill_decode_cache(w, SEED, q, DEV, slices=sample_kv)
+    kc, kd = _quantise(k, 0.5)
+    vc, vd = _quantise(v, 0.5)
+    del k, v
+    qd = q.to(DEV)
+    o, lse, keep, P = _decode(qd, kc, vc, w.tau, k_scale=0.5, v_scale=0.5)
+    heads = [(b, hk * 4 + g) for (b, hk) in sample_kv for g in range(4)]
+    rep = check_decode(qd, kd, vd, o, lse, keep, w.tau, P, heads=heads)
+    assert rep.heads == len(heads)
+    del kc, vc, kd, vd
+
+
+def test_decode_e4m3_rejects_bad_scales():
+    w, q, k, v = _small(1, 300)
+    kc, _ = _quantise(k, 1.0)
+    vc, _ = _quantise(v, 1.0)
+    with pytest.raises(mala.MalaError):
+        mala.mala_decode(q, kc, vc, w.tau, k_scale=0.0)
+    with pytest.raises(ValueError):
+        mala.mala_decode(q, kc, v, w.tau)            # mixed cache types

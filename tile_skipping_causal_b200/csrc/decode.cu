@@ -13,21 +13,43 @@
 // for tcgen05 (M >= 64), so scores and PV use warp-level mma.sync on
 // operands staged by TMA in 128-byte-swizzled shared memory.
 //
-// Roles (160 threads):
-//   warps 0-3  compute. QK^T: warp w scores keys [32w, 32w+32) of the tile
-//              for all rows; row maxima meet in shared memory; every warp
-//              then evaluates the same per-head decisions. PV: warp w owns
-//              output columns [32w, 32w+32) over all 128 keys.
-//   warp 4     TMA producer, polling: K tiles as far ahead as the K ring
-//              allows (independent of decisions), V tiles as decisions to
-//              retain arrive.
+// Roles (32 (W + 1) threads; W = 4 compute warps for bf16 caches, 8 for
+// e4m3 caches, whose per-tile work has more latency to hide):
+//   warps 0..W-1  compute. QK^T: warp w scores keys [w 128/W, (w+1) 128/W)
+//              of the tile for all rows; row maxima meet in shared memory;
+//              every warp then evaluates the same per-head decisions. PV:
+//              warp w owns output columns [w 128/W, (w+1) 128/W) over all
+//              128 keys. Warp 0 also issues each retained tile's V load, as
+//              soon as its V/P slot is free.
+//   warp W     TMA producer for K, in order: tiles as far ahead as the K
+//              ring allows (independent of decisions), blocking on the ring.
 // PV is deferred: a retained tile's P (bf16) and reference maxima wait in
 // one of two slots until the slot is needed again or the split ends, so the
-// V load issued after the vote overlaps the scoring of later tiles.
+// V load issued after the decision overlaps the scoring of later tiles.
+//
+// FP8 (e4m3) caches: tiles arrive as 128-byte rows (half the bytes, so the
+// K ring is twice as deep), and the mma.sync B fragments are built straight
+// from them, converting in registers (exactly: every e4m3 value is an f16):
+//   QK: the head dimension is visited in a permuted order, the same for the
+//       query fragments and K, chosen so that a thread's 32 values of a key
+//       row are 32 contiguous bytes (two 16-byte loads);
+//   PV: the output columns are permuted within each warp's 32, so that one
+//       4-byte load of a value row covers the thread's column in all four
+//       n-blocks; byte permutes pair consecutive keys for the fragments.
+// Both access patterns are free of bank conflicts under the 128-byte
+// swizzle. Scores and PV run as f16 mma.sync with the query and P in f16;
+// the cache scales are applied in fp32 (to the scores, and to O at the end).
 #include <math.h>
 
 #include "kernels.h"
 #include "ptx.cuh"
+
+#ifndef MALA_E4M3_CVT
+#define MALA_E4M3_CVT 1       // 0: convert with integer operations and an f16 multiply
+#endif
+#ifndef MALA_DECODE_BF16_WARPS
+#define MALA_DECODE_BF16_WARPS 4
+#endif
 
 namespace mala {
 
@@ -35,41 +57,61 @@ namespace {
 
 constexpr int kBK = 128;
 constexpr int kD = 128;
-constexpr int kNSK = 4;                 // K ring stages
+constexpr int kNSKMax = 8;              // K ring stages: 4 bf16 tiles, 8 e4m3 tiles
 constexpr int kNSV = 2;                 // V / P slots
-constexpr int kND = 4;                  // decision ring
-constexpr int kThreads = 160;
-constexpr uint32_t kTileBytes = kBK * kD * 2;
+constexpr uint32_t kTileBytes = kBK * kD * 2;   // bf16 tile (and staging tile)
 constexpr int kPStride = 136;           // bf16 per P row (128 + 8 padding)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 
 enum Bar {
-  kKFull = 0,                     // kNSK
-  kKEmpty = kKFull + kNSK,        // kNSK, 4 arrivals (one per compute warp)
-  kVFull = kKEmpty + kNSK,        // kNSV
+  kKFull = 0,                     // kNSKMax
+  kKEmpty = kKFull + kNSKMax,     // kNSKMax, 4 arrivals (one per compute warp)
+  kVFull = kKEmpty + kNSKMax,     // kNSV
   kSlotFree = kVFull + kNSV,      // kNSV, 4 arrivals
-  kDecFull = kSlotFree + kNSV,    // kND
-  kDecEmpty = kDecFull + kND,     // kND
-  kNumBars = kDecEmpty + kND
+  kNumBars = kSlotFree + kNSV
 };
 
+template <bool FP8>
 struct Smem {
+  static constexpr int kCW = FP8 ? 8 : MALA_DECODE_BF16_WARPS;          // compute warps
+  static constexpr int kThreads = 32 * (kCW + 1);                       // + the producer warp
+  static constexpr int kKPW = kBK / kCW;      // keys (scores) and value columns (PV) per compute warp
+  static constexpr int kNBW = kKPW / 8;       // mma n-blocks per compute warp
+  static constexpr int kNSK = FP8 ? 8 : 4;                              // K ring stages
+  static constexpr uint32_t kRing = FP8 ? kBK * kD : kTileBytes;        // bytes of a K / V ring tile
   static constexpr uint32_t kK = 0;
-  static constexpr uint32_t kV = kK + kNSK * kTileBytes;
-  static constexpr uint32_t kP = kV + kNSV * kTileBytes;                 // [kNSV][16][kPStride] bf16
+  static constexpr uint32_t kV = kK + kNSK * kRing;
+  static constexpr uint32_t kP = kV + kNSV * kRing;                     // [kNSV][16][kPStride] bf16 / f16
   static constexpr uint32_t kPendM = kP + kNSV * 16 * kPStride * 2;      // [kNSV][16] float
-  static constexpr uint32_t kPMax = kPendM + kNSV * 16 * 4;              // [2][4][16] float
-  static constexpr uint32_t kPSum = kPMax + 2 * 4 * 16 * 4;              // [2][4][16] float
-  static constexpr uint32_t kBars = kPSum + 2 * 4 * 16 * 4;
+  static constexpr uint32_t kPMax = kPendM + kNSV * 16 * 4;              // [2][kCW][16] float
+  static constexpr uint32_t kPSum = kPMax + 2 * kCW * 16 * 4;            // [2][kCW][16] float
+  static constexpr uint32_t kBars = kPSum + 2 * kCW * 16 * 4;
   static constexpr uint32_t kMisc = kBars + kNumBars * 8;               // misc words
   static constexpr uint32_t kEnd = kMisc + 64;
   static constexpr uint32_t kAlloc = kEnd + 1024;
 };
-static_assert(Smem::kAlloc <= 232448, "decode CTA exceeds shared memory");
+static_assert(Smem<false>::kAlloc <= 232448 && Smem<true>::kAlloc <= 232448, "decode CTA exceeds shared memory");
+static_assert(Smem<false>::kNSK <= kNSKMax && Smem<true>::kNSK <= kNSKMax, "K ring exceeds its barriers");
 
-__global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __grid_constant__ DecodeParams p) {
+// Four e4m3 values (bytes of w) to two f16x2 words: bytes 0, 1 -> lo and
+// 2, 3 -> hi, the lower byte in the lower half.
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+#if MALA_E4M3_CVT
+  lo = e4m3x2_to_f16x2(w & 0xFFFFu);
+  hi = e4m3x2_to_f16x2(w >> 16);
+#else
+  e4m3x4_to_f16x4(w, lo, hi);
+#endif
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kernel(const __grid_constant__ DecodeParams p) {
+  using Smem = mala::Smem<FP8>;
+  constexpr uint32_t kRing = Smem::kRing;
+  constexpr int kNSK = Smem::kNSK;
+  constexpr int kCW = Smem::kCW, kKPW = Smem::kKPW, kNBW = Smem::kNBW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -81,8 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
   float* sPSum = reinterpret_cast<float*>(smem + Smem::kPSum);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::kBars);
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + Smem::kMisc);
-  // misc[1] abort flag, misc[2..4] progress markers (producer / warp 0 /
-  // unused), misc[8..8+kND) decision ring
+  // misc[1] abort flag
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
   const int tid = threadIdx.x;
@@ -102,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
   if (tid == 0) {
     for (int x = 0; x < kNumBars; ++x) {
       uint32_t cnt = 1;
-      if ((x >= kKEmpty && x < kKEmpty + kNSK) || (x >= kSlotFree && x < kSlotFree + kNSV)) cnt = 4;
+      if ((x >= kKEmpty && x < kKEmpty + kNSKMax) || (x >= kSlotFree && x < kSlotFree + kNSV)) cnt = kCW;
       mbar_init(&bars[x], cnt);
     }
     for (int x = 1; x < 16; ++x) misc[x] = 0;
@@ -110,68 +151,21 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
   }
   __syncthreads();
 
-  if (warp == 4) {
-    // ===================== TMA producer (polling) =====================
+  if (warp == kCW) {
+    // ===================== K producer =====================
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_v);
-      int next_k = 0, next_d = 0, v_issued = 0, v_req = 0;
-      int vq[kND + kNSV];                // tiles waiting for a V load (ring)
-      uint64_t idle_since = global_timer_ns();
-      bool ok = true;
-      while (ok && (next_k < T || next_d < T || v_issued < v_req)) {
-        bool progress = false;
-        if (next_k < T) {
-          const int s = next_k % kNSK;
-          if (mbar_test(&bars[kKEmpty + s], ((next_k / kNSK) & 1) ^ 1)) {
-            mbar_expect_tx(&bars[kKFull + s], kTileBytes);
-            const int j = t1 - 1 - next_k;
-            for (int c = 0; c < 2; ++c)
-              tma_load_4d(sK + s * kTileBytes + c * 16384, &p.tm_k, &bars[kKFull + s], c * 64, hk,
-                          j * kBK, b);
-            ++next_k;
-            progress = true;
-          }
+      for (int t = 0; t < T; ++t) {
+        const int s = t % kNSK;
+        if (!mbar_wait(&bars[kKEmpty + s], ((t / kNSK) & 1) ^ 1, abort_flag, p.err, wait_tag(1, kKEmpty + s, t))) {
+          drain_pause_ns(50000);         // copies already issued land before the CTA exits
+          break;
         }
-        if (next_d < T) {
-          const int s = next_d % kND;
-          if (mbar_test(&bars[kDecFull + s], (next_d / kND) & 1)) {
-            const uint32_t keep = misc[8 + s];
-            mbar_arrive(&bars[kDecEmpty + s]);
-            if (keep) vq[v_req++ % (kND + kNSV)] = next_d;
-            ++next_d;
-            progress = true;
-          }
-        }
-        if (v_issued < v_req) {
-          const int s = v_issued % kNSV;
-          if (mbar_test(&bars[kSlotFree + s], ((v_issued / kNSV) & 1) ^ 1)) {
-            const int t = vq[v_issued % (kND + kNSV)];
-            const int j = t1 - 1 - t;
-            mbar_expect_tx(&bars[kVFull + s], kTileBytes);
-            for (int c = 0; c < 2; ++c)
-              tma_load_4d(sV + s * kTileBytes + c * 16384, &p.tm_v, &bars[kVFull + s], c * 64, hk,
-                          j * kBK, b);
-            ++v_issued;
-            progress = true;
-          }
-        }
-        misc[2] = (static_cast<uint32_t>(next_k) << 20) | (static_cast<uint32_t>(next_d) << 10) | v_issued;
-        if (progress) {
-          idle_since = global_timer_ns();
-        } else if (*abort_flag) {
-          ok = false;
-        } else if (global_timer_ns() - idle_since > kWaitLimitNs) {
-          *abort_flag = 1;
-          if (atomicCAS(p.err, 0, kErrTimeout) == 0) {
-            p.err[1] = wait_tag(1, 0xff, next_d);
-            p.err[2] = static_cast<int>(blockIdx.x);
-            for (int x = 0; x < 3; ++x) p.err[4 + x] = misc[2 + x];
-          }
-          ok = false;
-        }
+        mbar_expect_tx(&bars[kKFull + s], kRing);
+        const int j = t1 - 1 - t;
+        for (int c = 0; c < (FP8 ? 1 : 2); ++c)
+          tma_load_4d(sK + s * kRing + c * 16384, &p.tm_k, &bars[kKFull + s], c * 64, hk, j * kBK, b);
       }
-      if (!ok) drain_pause_ns(50000);
     }
   } else {
     // ===================== compute warps =====================
@@ -182,8 +176,10 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
     const int h_lo = has_lo ? p.group_heads[hk][row_lo] : 0;
     const int h_hi = has_hi ? p.group_heads[hk][row_hi] : 0;
     const float thr2 = p.log2_tau - log2f(static_cast<float>(p.Nk));   // log2(tau / L_0)
+    if (warp == 0 && lane == 0) tma_prefetch_desc(&p.tm_v);
 
-    // query A fragments for the 8 k-steps over d = 128
+    // query A fragments for the 8 k-steps over d = 128; FP8 caches: k-step
+    // kk, fragment column 2tq + e (+ 8) holds d = 32tq + 4kk + e (+ 2)
     uint32_t qa[8][4];
     {
       const uint32_t* qlo = reinterpret_cast<const uint32_t*>(
@@ -192,19 +188,25 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
           reinterpret_cast<const __nv_bfloat16*>(p.q) + b * p.q_sb + h_hi * p.q_sh);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        qa[kk][0] = has_lo ? qlo[(16 * kk + 2 * tq) >> 1] : 0u;
-        qa[kk][1] = has_hi ? qhi[(16 * kk + 2 * tq) >> 1] : 0u;
-        qa[kk][2] = has_lo ? qlo[(16 * kk + 8 + 2 * tq) >> 1] : 0u;
-        qa[kk][3] = has_hi ? qhi[(16 * kk + 8 + 2 * tq) >> 1] : 0u;
+        const int w0 = FP8 ? 16 * tq + 2 * kk : (16 * kk + 2 * tq) >> 1;
+        const int w1 = FP8 ? w0 + 1 : w0 + 4;
+        qa[kk][0] = has_lo ? qlo[w0] : 0u;
+        qa[kk][1] = has_hi ? qhi[w0] : 0u;
+        qa[kk][2] = has_lo ? qlo[w1] : 0u;
+        qa[kk][3] = has_hi ? qhi[w1] : 0u;
+        if constexpr (FP8) {
+#pragma unroll
+          for (int x = 0; x < 4; ++x) qa[kk][x] = bf16x2_to_f16x2(qa[kk][x]);
+        }
       }
     }
 
     float m2_lo = -INFINITY, m2_hi = -INFINITY;   // reference maxima (log2 units)
     float l_lo = 0.0f, l_hi = 0.0f;               // normalisation sums
     float om_lo = -INFINITY, om_hi = -INFINITY;   // reference of the O accumulator rows
-    float o[4][4];
+    float o[kNBW][4];
 #pragma unroll
-    for (int nb = 0; nb < 4; ++nb)
+    for (int nb = 0; nb < kNBW; ++nb)
 #pragma unroll
       for (int x = 0; x < 4; ++x) o[nb][x] = 0.0f;
     int kc = 0, pv_done = 0;                     // retained tiles, PVs executed
@@ -216,9 +218,9 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
     auto fold_sums = [&](int par) {
       float a = 0.0f, c = 0.0f;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        a += sPSum[(par * 4 + w) * 16 + row_lo];
-        c += sPSum[(par * 4 + w) * 16 + row_hi];
+      for (int w = 0; w < kCW; ++w) {
+        a += sPSum[(par * kCW + w) * 16 + row_lo];
+        c += sPSum[(par * kCW + w) * 16 + row_hi];
       }
       l_lo += a;
       l_hi += c;
@@ -236,13 +238,13 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
         om_lo = pm_lo;
         om_hi = pm_hi;
 #pragma unroll
-        for (int nb = 0; nb < 4; ++nb) {
+        for (int nb = 0; nb < kNBW; ++nb) {
           o[nb][0] *= f_lo; o[nb][1] *= f_lo;
           o[nb][2] *= f_hi; o[nb][3] *= f_hi;
         }
         const uint32_t* prow_lo = reinterpret_cast<const uint32_t*>(sP + (s * 16 + row_lo) * kPStride);
         const uint32_t* prow_hi = reinterpret_cast<const uint32_t*>(sP + (s * 16 + row_hi) * kPStride);
-        const uint32_t vbase = sVa + s * kTileBytes;
+        const uint32_t vbase = sVa + s * kRing;
         const int mi = lane >> 3, rr = lane & 7;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -250,15 +252,37 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
           const uint32_t a1 = prow_hi[(16 * kk + 2 * tq) >> 1];
           const uint32_t a2 = prow_lo[(16 * kk + 8 + 2 * tq) >> 1];
           const uint32_t a3 = prow_hi[(16 * kk + 8 + 2 * tq) >> 1];
+          if constexpr (FP8) {
+            // n-block nb, fragment column g is value column kKPW w + kNBW g + nb:
+            // bytes [kKPW w + kNBW g, + kNBW) of the rows of keys 16kk + 2tq
+            // (+1, +8, +9), paired across consecutive keys
+            const int cb = kKPW * warp + kNBW * g;
+            uint32_t r[4];
 #pragma unroll
-          for (int nb = 0; nb < 4; nb += 2) {
-            // matrices: (keys 16kk+[0,8) | +8, cols 32w+8nb) then (cols +8)
-            const int key = 16 * kk + ((mi & 1) << 3) + rr;
-            const int col = 32 * warp + 8 * (nb + (mi >> 1));
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_trans(sw128_addr(vbase, key, col), b0, b1, b2, b3);
-            mma_bf16_16816(o[nb], a0, a1, a2, a3, b0, b1);
-            mma_bf16_16816(o[nb + 1], a0, a1, a2, a3, b2, b3);
+            for (int x = 0; x < 4; ++x) {
+              const uint32_t a = sw128_addr_b8(vbase, 16 * kk + 2 * tq + (x & 1) + 8 * (x >> 1), cb >> 4) + (cb & 15);
+              r[x] = kNBW == 4 ? ld_shared_u32(a) : ld_shared_u16(a);
+            }
+            uint32_t b0[kNBW], b1[kNBW];
+            e4m3x4_to_f16(__byte_perm(r[0], r[1], 0x5140), b0[0], b0[1]);
+            e4m3x4_to_f16(__byte_perm(r[2], r[3], 0x5140), b1[0], b1[1]);
+            if constexpr (kNBW == 4) {
+              e4m3x4_to_f16(__byte_perm(r[0], r[1], 0x7362), b0[2], b0[3]);
+              e4m3x4_to_f16(__byte_perm(r[2], r[3], 0x7362), b1[2], b1[3]);
+            }
+#pragma unroll
+            for (int nb = 0; nb < kNBW; ++nb) mma_f16_16816(o[nb], a0, a1, a2, a3, b0[nb], b1[nb]);
+          } else {
+#pragma unroll
+            for (int nb = 0; nb < kNBW; nb += 2) {
+              // matrices: (keys 16kk+[0,8) | +8, cols 32w+8nb) then (cols +8)
+              const int key = 16 * kk + ((mi & 1) << 3) + rr;
+              const int col = kKPW * warp + 8 * (nb + (mi >> 1));
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4_trans(sw128_addr(vbase, key, col), b0, b1, b2, b3);
+              mma_bf16_16816(o[nb], a0, a1, a2, a3, b0, b1);
+              mma_bf16_16816(o[nb + 1], a0, a1, a2, a3, b2, b3);
+            }
           }
         }
       }
@@ -273,35 +297,57 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
       const int ks = t % kNSK;
       const bool okk = __all_sync(0xffffffffu, mbar_wait(&bars[kKFull + ks], (t / kNSK) & 1, abort_flag, p.err,
                                                          wait_tag(0, kKFull + ks, t)));
-      float sacc[4][4];
+      float sacc[kNBW][4];
 #pragma unroll
-      for (int nb = 0; nb < 4; ++nb)
+      for (int nb = 0; nb < kNBW; ++nb)
 #pragma unroll
         for (int x = 0; x < 4; ++x) sacc[nb][x] = 0.0f;
       if (okk) {
-        const uint32_t kbase = sKa + ks * kTileBytes;
-        const int mi = lane >> 3, rr = lane & 7;
+        const uint32_t kbase = sKa + ks * kRing;
+        if constexpr (FP8) {
+          // n-block nb, fragment column g is key kKPW w + 8nb + g; k-step kk
+          // takes bytes 4kk .. 4kk + 3 of its bytes [32tq, 32tq + 32)
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+          for (int nb = 0; nb < kNBW; ++nb) {
+            const int key = kKPW * warp + 8 * nb + g;
+            uint32_t w[8];
+            ld_shared_v4(sw128_addr_b8(kbase, key, 2 * tq), w[0], w[1], w[2], w[3]);
+            ld_shared_v4(sw128_addr_b8(kbase, key, 2 * tq + 1), w[4], w[5], w[6], w[7]);
 #pragma unroll
-          for (int nb = 0; nb < 4; nb += 2) {
-            // matrices: (keys 32w+8nb+[0,8), d 16kk | +8), then keys +8
-            const int key = 32 * warp + 8 * (nb + (mi >> 1)) + rr;
-            const int d0 = 16 * kk + ((mi & 1) << 3);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(sw128_addr(kbase, key, d0), b0, b1, b2, b3);
-            mma_bf16_16816(sacc[nb], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
-            mma_bf16_16816(sacc[nb + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
+            for (int kk = 0; kk < 8; ++kk) {
+              uint32_t b0, b1;
+              e4m3x4_to_f16(w[kk], b0, b1);
+              mma_f16_16816(sacc[nb], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
+            }
+          }
+#pragma unroll
+          for (int nb = 0; nb < kNBW; ++nb)
+#pragma unroll
+            for (int x = 0; x < 4; ++x) sacc[nb][x] *= p.k_scale;
+        } else {
+          const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+            for (int nb = 0; nb < kNBW; nb += 2) {
+              // matrices: (keys kKPW w+8nb+[0,8), d 16kk | +8), then keys +8
+              const int key = kKPW * warp + 8 * (nb + (mi >> 1)) + rr;
+              const int d0 = 16 * kk + ((mi & 1) << 3);
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4(sw128_addr(kbase, key, d0), b0, b1, b2, b3);
+              mma_bf16_16816(sacc[nb], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
+              mma_bf16_16816(sacc[nb + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
+            }
           }
         }
       }
       // keys past the cache end (last tile only) do not exist
       float mx_lo = -INFINITY, mx_hi = -INFINITY;
 #pragma unroll
-      for (int nb = 0; nb < 4; ++nb) {
+      for (int nb = 0; nb < kNBW; ++nb) {
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-          const int key = j * kBK + 32 * warp + 8 * nb + 2 * tq + x;
+          const int key = j * kBK + kKPW * warp + 8 * nb + 2 * tq + x;
           if (key >= p.Nk) {
             sacc[nb][x] = -INFINITY;
             sacc[nb][2 + x] = -INFINITY;
@@ -315,21 +361,21 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
       mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
       mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
       if (tq == 0) {
-        sPMax[((t & 1) * 4 + warp) * 16 + row_lo] = mx_lo;
-        sPMax[((t & 1) * 4 + warp) * 16 + row_hi] = mx_hi;
+        sPMax[((t & 1) * kCW + warp) * 16 + row_lo] = mx_lo;
+        sPMax[((t & 1) * kCW + warp) * 16 + row_hi] = mx_hi;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kKEmpty + ks]);
       // one barrier per tile; the OR of the abort flag keeps every warp's exit in step
-      if (bar_or(1, 128, *abort_flag != 0)) break;
+      if (bar_or(1, 32 * kCW, *abort_flag != 0)) break;
 
       // previous tile's sums, this tile's maxima, per-head decisions
       if (prev_any) fold_sums((t - 1) & 1);
       float tm_lo = -INFINITY, tm_hi = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        tm_lo = fmaxf(tm_lo, sPMax[((t & 1) * 4 + w) * 16 + row_lo]);
-        tm_hi = fmaxf(tm_hi, sPMax[((t & 1) * 4 + w) * 16 + row_hi]);
+      for (int w = 0; w < kCW; ++w) {
+        tm_lo = fmaxf(tm_lo, sPMax[((t & 1) * kCW + w) * 16 + row_lo]);
+        tm_hi = fmaxf(tm_hi, sPMax[((t & 1) * kCW + w) * 16 + row_hi]);
       }
       const float tm2_lo = tm_lo * kLog2e, tm2_hi = tm_hi * kLog2e;
       const bool keep_lo = has_lo && (l_lo == 0.0f || tm2_lo - (m2_lo + lg2_approx(l_lo)) >= thr2);
@@ -346,15 +392,6 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
           mw_lo = mw_hi = 0;
         }
       }
-      // publish the decision to the producer
-      if (warp == 0 && lane == 0) {
-        const int s = t % kND;
-        if (mbar_wait(&bars[kDecEmpty + s], ((t / kND) & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty + s, t))) {
-          misc[8 + s] = any ? 1u : 0u;
-          mbar_arrive(&bars[kDecFull + s]);
-        }
-        misc[3] = 0x10000u | t;
-      }
       prev_any = any;
       if (!any) continue;
 
@@ -369,37 +406,44 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
       }
       // P = 2^(s log2e - m2) for retaining rows, 0 otherwise
       float ps_lo = 0.0f, ps_hi = 0.0f;
-      uint32_t pk_lo[4], pk_hi[4];
+      uint32_t pk_lo[kNBW], pk_hi[kNBW];
 #pragma unroll
-      for (int nb = 0; nb < 4; ++nb) {
+      for (int nb = 0; nb < kNBW; ++nb) {
         const float a0 = keep_lo ? ex2_approx(fmaf(sacc[nb][0], kLog2e, -m2_lo)) : 0.0f;
         const float a1 = keep_lo ? ex2_approx(fmaf(sacc[nb][1], kLog2e, -m2_lo)) : 0.0f;
         const float c0 = keep_hi ? ex2_approx(fmaf(sacc[nb][2], kLog2e, -m2_hi)) : 0.0f;
         const float c1 = keep_hi ? ex2_approx(fmaf(sacc[nb][3], kLog2e, -m2_hi)) : 0.0f;
         ps_lo += a0 + a1;
         ps_hi += c0 + c1;
-        pk_lo[nb] = pack_bf16x2(a0, a1);
-        pk_hi[nb] = pack_bf16x2(c0, c1);
+        pk_lo[nb] = FP8 ? pack_f16x2(a0, a1) : pack_bf16x2(a0, a1);
+        pk_hi[nb] = FP8 ? pack_f16x2(c0, c1) : pack_bf16x2(c0, c1);
       }
       ps_lo += __shfl_xor_sync(0xffffffffu, ps_lo, 1);
       ps_lo += __shfl_xor_sync(0xffffffffu, ps_lo, 2);
       ps_hi += __shfl_xor_sync(0xffffffffu, ps_hi, 1);
       ps_hi += __shfl_xor_sync(0xffffffffu, ps_hi, 2);
       if (tq == 0) {
-        sPSum[((t & 1) * 4 + warp) * 16 + row_lo] = ps_lo;
-        sPSum[((t & 1) * 4 + warp) * 16 + row_hi] = ps_hi;
+        sPSum[((t & 1) * kCW + warp) * 16 + row_lo] = ps_lo;
+        sPSum[((t & 1) * kCW + warp) * 16 + row_hi] = ps_hi;
       }
       // a free P/V slot: run the oldest pending PV when both are taken
       if (kc - pv_done == kNSV) do_pv();
       const int s = kc % kNSV;
-      mbar_wait(&bars[kSlotFree + s], ((kc / kNSV) & 1) ^ 1, abort_flag, p.err, wait_tag(0, kSlotFree + s, kc));
+      const bool slot_ok = mbar_wait(&bars[kSlotFree + s], ((kc / kNSV) & 1) ^ 1, abort_flag, p.err,
+                                     wait_tag(0, kSlotFree + s, kc));
+      if (warp == 0 && lane == 0 && slot_ok) {
+        // every warp has finished the slot's previous PV: load this tile's V
+        mbar_expect_tx(&bars[kVFull + s], kRing);
+        for (int c = 0; c < (FP8 ? 1 : 2); ++c)
+          tma_load_4d(sV + s * kRing + c * 16384, &p.tm_v, &bars[kVFull + s], c * 64, hk, j * kBK, b);
+      }
       {
         uint32_t* prow_lo = reinterpret_cast<uint32_t*>(sP + (s * 16 + row_lo) * kPStride);
         uint32_t* prow_hi = reinterpret_cast<uint32_t*>(sP + (s * 16 + row_hi) * kPStride);
 #pragma unroll
-        for (int nb = 0; nb < 4; ++nb) {
-          prow_lo[(32 * warp + 8 * nb + 2 * tq) >> 1] = pk_lo[nb];
-          prow_hi[(32 * warp + 8 * nb + 2 * tq) >> 1] = pk_hi[nb];
+        for (int nb = 0; nb < kNBW; ++nb) {
+          prow_lo[(kKPW * warp + 8 * nb + 2 * tq) >> 1] = pk_lo[nb];
+          prow_hi[(kKPW * warp + 8 * nb + 2 * tq) >> 1] = pk_hi[nb];
         }
         if (warp == 0 && tq == 0) {
           sPendM[s * 16 + row_lo] = has_lo ? m2_lo : 0.0f;
@@ -410,25 +454,42 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
     }
 
     // drain the deferred PVs; the last barrier makes every warp's P and sums visible
-    if (!bar_or(1, 128, *abort_flag != 0)) {
+    if (!bar_or(1, 32 * kCW, *abort_flag != 0)) {
       while (pv_done < kc) do_pv();
       if (prev_any) fold_sums((T - 1) & 1);
       // outputs: rows < G of this warp's 32 columns
-      const float inv_lo = l_lo > 0.0f ? 1.0f / l_lo : 0.0f;
-      const float inv_hi = l_hi > 0.0f ? 1.0f / l_hi : 0.0f;
+      // FP8 caches: the value scale folds into the normalisation
+      const float vs = FP8 ? p.v_scale : 1.0f;
+      const float inv_lo = l_lo > 0.0f ? vs / l_lo : 0.0f;
+      const float inv_hi = l_hi > 0.0f ? vs / l_hi : 0.0f;
       const float z_lo = (m2_lo + log2f(l_lo)) * kLn2;
       const float z_hi = (m2_hi + log2f(l_hi)) * kLn2;
+      // column pairs (c, c + 1) this thread writes, c = col[i], with rows lo
+      // (vl) and hi (vh): bf16 caches: n-block i, c = kKPW w + 8i + 2tq. FP8
+      // caches (n-block nb, fragment column n is kKPW w + kNBW n + nb): the
+      // thread's columns are kKPW w + 2 kNBW tq + e, e < 2 kNBW, from
+      // o[e % kNBW][e / kNBW]
+      int col[kNBW];
+      float vl[kNBW][2], vh[kNBW][2];
+#pragma unroll
+      for (int i = 0; i < kNBW; ++i) {
+        const int nb = FP8 ? (2 * i) % kNBW : i, x = FP8 ? (2 * i) / kNBW : 0;
+        col[i] = FP8 ? kKPW * warp + 2 * kNBW * tq + 2 * i : kKPW * warp + 8 * i + 2 * tq;
+        vl[i][0] = FP8 ? o[nb][x] : o[nb][0];
+        vl[i][1] = FP8 ? o[nb + 1][x] : o[nb][1];
+        vh[i][0] = FP8 ? o[nb][2 + x] : o[nb][2];
+        vh[i][1] = FP8 ? o[nb + 1][2 + x] : o[nb][3];
+      }
       if (P == 1) {
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.o);
 #pragma unroll
-        for (int nb = 0; nb < 4; ++nb) {
-          const int col = 32 * warp + 8 * nb + 2 * tq;
+        for (int i = 0; i < kNBW; ++i) {
           if (has_lo)
-            *reinterpret_cast<uint32_t*>(out + b * p.o_sb + h_lo * p.o_sh + col) =
-                pack_bf16x2(o[nb][0] * inv_lo, o[nb][1] * inv_lo);
+            *reinterpret_cast<uint32_t*>(out + b * p.o_sb + h_lo * p.o_sh + col[i]) =
+                pack_bf16x2(vl[i][0] * inv_lo, vl[i][1] * inv_lo);
           if (has_hi)
-            *reinterpret_cast<uint32_t*>(out + b * p.o_sb + h_hi * p.o_sh + col) =
-                pack_bf16x2(o[nb][2] * inv_hi, o[nb][3] * inv_hi);
+            *reinterpret_cast<uint32_t*>(out + b * p.o_sb + h_hi * p.o_sh + col[i]) =
+                pack_bf16x2(vh[i][0] * inv_hi, vh[i][1] * inv_hi);
         }
         if (warp == 0 && tq == 0) {
           if (has_lo) p.lse[b * p.Hq + h_lo] = z_lo;
@@ -436,15 +497,14 @@ __global__ void __launch_bounds__(kThreads, 1) mala_decode_split_kernel(const __
         }
       } else {
 #pragma unroll
-        for (int nb = 0; nb < 4; ++nb) {
-          const int col = 32 * warp + 8 * nb + 2 * tq;
+        for (int i = 0; i < kNBW; ++i) {
           if (has_lo) {
-            float2* dst = reinterpret_cast<float2*>(p.part_o + ((static_cast<int64_t>(b) * p.Hq + h_lo) * P + split) * kD + col);
-            *dst = make_float2(o[nb][0] * inv_lo, o[nb][1] * inv_lo);
+            float2* dst = reinterpret_cast<float2*>(p.part_o + ((static_cast<int64_t>(b) * p.Hq + h_lo) * P + split) * kD + col[i]);
+            *dst = make_float2(vl[i][0] * inv_lo, vl[i][1] * inv_lo);
           }
           if (has_hi) {
-            float2* dst = reinterpret_cast<float2*>(p.part_o + ((static_cast<int64_t>(b) * p.Hq + h_hi) * P + split) * kD + col);
-            *dst = make_float2(o[nb][2] * inv_hi, o[nb][3] * inv_hi);
+            float2* dst = reinterpret_cast<float2*>(p.part_o + ((static_cast<int64_t>(b) * p.Hq + h_hi) * P + split) * kD + col[i]);
+            *dst = make_float2(vh[i][0] * inv_hi, vh[i][1] * inv_hi);
           }
         }
         if (warp == 0 && tq == 0) {
@@ -487,15 +547,22 @@ __global__ void __launch_bounds__(128) mala_decode_combine_kernel(const __grid_c
 
 }  // namespace
 
-size_t decode_smem_bytes() { return Smem::kAlloc; }
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream) {
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hkv * p.num_splits;
   if (grid == 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(mala_decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(Smem::kAlloc));
-  if (e != cudaSuccess) return e;
-  mala_decode_split_kernel<<<grid, kThreads, Smem::kAlloc, stream>>>(p);
+  cudaError_t e;
+  if (p.kv_fp8) {
+    e = cudaFuncSetAttribute(mala_decode_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(Smem<true>::kAlloc));
+    if (e != cudaSuccess) return e;
+    mala_decode_split_kernel<true><<<grid, Smem<true>::kThreads, Smem<true>::kAlloc, stream>>>(p);
+  } else {
+    e = cudaFuncSetAttribute(mala_decode_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(Smem<false>::kAlloc));
+    if (e != cudaSuccess) return e;
+    mala_decode_split_kernel<false><<<grid, Smem<false>::kThreads, Smem<false>::kAlloc, stream>>>(p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess || p.num_splits == 1) return e;
   mala_decode_combine_kernel<<<p.B * p.Hq, kD, 0, stream>>>(p);

@@ -83,12 +83,13 @@ struct DecodeParams {
   int64_t q_sb, q_sh, o_sb, o_sh;
   int B, Hq, Hkv, Nk, nKB, mask_words, num_splits;
   float log2_tau;
+  int kv_fp8;           // K and V cache in e4m3 (tm_k / tm_v are then byte maps)
+  float k_scale, v_scale;   // e4m3 cache scales (value = code * scale)
   uint8_t group_size[kMaxKvHeads];
   uint8_t group_heads[kMaxKvHeads][kMaxGroup];
 };
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
-size_t decode_smem_bytes();
 
 // Backward (bf16, d = 128, B_q = B_k = 128, N_q <= N_k bottom-right aligned).
 struct BwdParams {

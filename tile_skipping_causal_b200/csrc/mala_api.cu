@@ -76,6 +76,23 @@ int make_map_bf16(CUtensorMap* map, const void* ptr, int64_t B, int64_t N, int64
   return MALA_OK;
 }
 
+// 4-D byte view {d, heads, seq, batch} of an e4m3 [B, N, H, d] tensor, box
+// {128, 1, rows, 1}: one 128-byte row per key, 128-byte swizzle.
+int make_map_u8(CUtensorMap* map, const void* ptr, int64_t B, int64_t N, int64_t H, int64_t d,
+                const int64_t* st, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MALA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)st[2], (cuuint64_t)st[1], (cuuint64_t)st[0]};
+  cuuint32_t box[4] = {128, 1, (cuuint32_t)rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MALA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MALA_OK;
+}
+
 // Device address of the error block on the current device (looked up once
 // per device; calls from several host threads are serialised here).
 int* device_error_ptr() {
@@ -480,11 +497,35 @@ int decode_check(const mala_decode_args* a, int* nKB_out) {
   const int nKB = static_cast<int>((a->seqlen_k + 127) / 128);
   if (a->num_splits < 0 || a->num_splits > nKB)
     return fail(MALA_ERR_INVALID_ARG, "num_splits %d outside [0, %d]", a->num_splits, nKB);
+  if (a->kv_dtype != MALA_BF16 && a->kv_dtype != MALA_FP8_E4M3)
+    return fail(MALA_ERR_INVALID_ARG, "kv_dtype %d is neither MALA_BF16 nor MALA_FP8_E4M3", a->kv_dtype);
+  const bool fp8 = a->kv_dtype == MALA_FP8_E4M3;
+  if (fp8 && !(a->k_scale > 0.0f && a->k_scale < INFINITY && a->v_scale > 0.0f && a->v_scale < INFINITY))
+    return fail(MALA_ERR_INVALID_ARG, "e4m3 cache scales must be positive and finite");
+  const int64_t kes = fp8 ? 1 : 2;
   if ((rc = check_tensor("q", a->q, a->q_stride, 2, 128, a->heads_q))) return rc;
-  if ((rc = check_tensor("k", a->k, a->k_stride, 2, 128, a->heads_kv))) return rc;
-  if ((rc = check_tensor("v", a->v, a->v_stride, 2, 128, a->heads_kv))) return rc;
+  if ((rc = check_tensor("k", a->k, a->k_stride, kes, 128, a->heads_kv))) return rc;
+  if ((rc = check_tensor("v", a->v, a->v_stride, kes, 128, a->heads_kv))) return rc;
   if ((rc = check_tensor("o", a->o, a->o_stride, 2, 128, a->heads_q))) return rc;
   *nKB_out = nKB;
+  return MALA_OK;
+}
+
+// K / V cache tensor maps, element type and scales of a decode call.
+int decode_cache_maps(const mala_decode_args* a, mala::DecodeParams* p) {
+  int rc;
+  if (a->kv_dtype == MALA_FP8_E4M3) {
+    if ((rc = make_map_u8(&p->tm_k, a->k, a->batch, a->seqlen_k, a->heads_kv, 128, a->k_stride, 128))) return rc;
+    if ((rc = make_map_u8(&p->tm_v, a->v, a->batch, a->seqlen_k, a->heads_kv, 128, a->v_stride, 128))) return rc;
+    p->kv_fp8 = 1;
+    p->k_scale = a->k_scale;
+    p->v_scale = a->v_scale;
+  } else {
+    if ((rc = make_map_bf16(&p->tm_k, a->k, a->batch, a->seqlen_k, a->heads_kv, 128, a->k_stride, 128))) return rc;
+    if ((rc = make_map_bf16(&p->tm_v, a->v, a->batch, a->seqlen_k, a->heads_kv, 128, a->v_stride, 128))) return rc;
+    p->kv_fp8 = 0;
+    p->k_scale = p->v_scale = 1.0f;
+  }
   return MALA_OK;
 }
 
@@ -541,8 +582,7 @@ int mala_decode(mala_decode_args* a, void* workspace, size_t ws_bytes, void* str
       return fail(MALA_ERR_UNSUPPORTED, "more than %d query heads share KV head %d", mala::kMaxGroup, hk);
     p.group_heads[hk][p.group_size[hk]++] = static_cast<uint8_t>(h);
   }
-  if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, a->seqlen_k, a->heads_kv, 128, a->k_stride, 128))) return rc;
-  if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, a->seqlen_k, a->heads_kv, 128, a->v_stride, 128))) return rc;
+  if ((rc = decode_cache_maps(a, &p))) return rc;
   p.err = device_error_ptr();
   if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
   p.q = a->q;
@@ -643,8 +683,7 @@ extern "C" int mala_decode_noalloc(mala_decode_args* a, void* stream_) {
       return fail(MALA_ERR_UNSUPPORTED, "more than %d query heads share KV head %d", mala::kMaxGroup, hk);
     p.group_heads[hk][p.group_size[hk]++] = static_cast<uint8_t>(h);
   }
-  if ((rc = make_map_bf16(&p.tm_k, a->k, a->batch, a->seqlen_k, a->heads_kv, 128, a->k_stride, 128))) return rc;
-  if ((rc = make_map_bf16(&p.tm_v, a->v, a->batch, a->seqlen_k, a->heads_kv, 128, a->v_stride, 128))) return rc;
+  if ((rc = decode_cache_maps(a, &p))) return rc;
   p.err = device_error_ptr();
   if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
   p.q = a->q;

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -327,6 +328,75 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       "{%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two bf16 (low, high half) to two f16 through fp32.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  return pack_f16x2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+
+// Two e4m3 values (byte 0 -> low half, byte 1 -> high half) to f16x2; every
+// e4m3 value is exactly representable in f16.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "r"(two_bytes));
+  return r;
+}
+
+// Four e4m3 values (bytes 0..3 of w) to two f16x2 words (bytes 0, 1 -> lo;
+// 2, 3 -> hi) with integer operations and one f16 multiply: each byte's
+// exponent and mantissa bits are placed at the f16 exponent / mantissa
+// positions (bits 13..7), which reads as 2^-8 times the e4m3 value (its bias
+// 7 against f16's 15; subnormals map to f16 subnormals), with the sign at
+// bit 15; the multiply by 2^8 is then exact.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t a = __byte_perm(w, 0u, 0x4140);   // [0, b1, 0, b0]
+  const uint32_t c = __byte_perm(w, 0u, 0x4342);   // [0, b3, 0, b2]
+  const uint32_t a16 = ((a << 7) & 0x3F803F80u) | ((a << 8) & 0x80008000u);
+  const uint32_t c16 = ((c << 7) & 0x3F803F80u) | ((c << 8) & 0x80008000u);
+  const __half2 k256 = __half2(__ushort_as_half(0x5C00), __ushort_as_half(0x5C00));
+  __half2 x = __hmul2(*reinterpret_cast<const __half2*>(&a16), k256);
+  __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&c16), k256);
+  lo = *reinterpret_cast<uint32_t*>(&x);
+  hi = *reinterpret_cast<uint32_t*>(&y);
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// zero-extended
+__device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr)
+               : "memory");
+}
+
+// Byte address of the 16-byte unit u (bytes [16u, 16u + 16)) of row `row`
+// in a tile of 128-byte rows loaded by TMA with 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw128_addr_b8(uint32_t base, int row, int u) {
+  return base + row * 128 + ((u ^ (row & 7)) << 4);
 }
 
 // Byte address of the 16-byte unit holding elements [d0, d0 + 8) of row

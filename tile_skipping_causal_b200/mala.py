@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "lib", "libmala.so")
 
 MALA_OK, MALA_ERR_INVALID_ARG, MALA_ERR_UNSUPPORTED, MALA_ERR_WORKSPACE, MALA_ERR_CUDA, \
     MALA_ERR_TIMEOUT = range(6)
-MALA_BF16, MALA_FP32 = 0, 1
+MALA_BF16, MALA_FP32, MALA_FP8_E4M3 = 0, 1, 2
 MALA_CAUSAL, MALA_DECODE = 0, 1
 
 _i64x3 = ctypes.c_int64 * 3
@@ -64,6 +64,7 @@ class DecodeArgs(ctypes.Structure):
         ("q_stride", _i64x3), ("k_stride", _i64x3), ("v_stride", _i64x3), ("o_stride", _i64x3),
         ("q_to_kv", ctypes.c_void_p), ("block_k", ctypes.c_int32), ("tau", ctypes.c_float),
         ("dtype", ctypes.c_int32), ("num_splits", ctypes.c_int32), ("stats", ctypes.c_void_p),
+        ("kv_dtype", ctypes.c_int32), ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
     ]
 
 
@@ -325,12 +326,22 @@ def mala_bwd(q, k, v, o, do, lse, tau: float, keep_mask=None, block_q: int = 128
     return dq, dk, dv, bwd_keep_mask
 
 
+def _decode_cache(a, k, v, k_scale, v_scale):
+    """Cache element type: bf16, or e4m3 codes with their scales."""
+    fp8 = (k.dtype == torch.float8_e4m3fn, v.dtype == torch.float8_e4m3fn)
+    if fp8[0] != fp8[1]:
+        raise ValueError("k and v caches must have the same element type")
+    a.kv_dtype = MALA_FP8_E4M3 if fp8[0] else MALA_BF16
+    a.k_scale, a.v_scale = float(k_scale), float(v_scale)
+
+
 def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *, o=None,
                 lse=None, keep_mask=None, with_mask: bool = True, stats=None, q_to_kv=None,
-                stream=None, workspace=None):
-    """Single-token decoding. q [B, 1, Hq, d]; k/v cache [B, Nk, Hkv, d].
-    Returns (o, lse [B, Hq], keep_mask words [B, Hq, ceil(T/32)] or None,
-    num_splits used)."""
+                stream=None, workspace=None, k_scale: float = 1.0, v_scale: float = 1.0):
+    """Single-token decoding. q [B, 1, Hq, d] bf16; k/v cache [B, Nk, Hkv, d]
+    in bf16, or torch.float8_e4m3fn codes whose values are code * k_scale and
+    code * v_scale. Returns (o, lse [B, Hq], keep_mask words
+    [B, Hq, ceil(T/32)] or None, num_splits used)."""
     lib = load_library()
     _require_cuda(q, k, v)
     B, _, Hq, d = q.shape
@@ -352,6 +363,7 @@ def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *,
     a.dtype = _dtype_code(q)
     a.num_splits = int(num_splits)
     a.stats = _ptr(stats)
+    _decode_cache(a, k, v, k_scale, v_scale)
     ws_n = lib.mala_decode_workspace_size(ctypes.byref(a))
     own_ws = workspace is None or workspace.numel() < ws_n
     if own_ws:
@@ -365,7 +377,7 @@ def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *,
 
 def mala_decode_noalloc(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *, o=None,
                         lse=None, keep_mask=None, with_mask: bool = True, stats=None, q_to_kv=None,
-                        stream=None):
+                        stream=None, k_scale: float = 1.0, v_scale: float = 1.0):
     """mala_decode without a workspace: the library keeps the split partials
     in its own built-in device buffer (for callers that cannot allocate;
     calls that overlap on the GPU race on that buffer). Returns the same
@@ -391,6 +403,7 @@ def mala_decode_noalloc(q, k, v, tau: float, block_k: int = 128, num_splits: int
     a.dtype = _dtype_code(q)
     a.num_splits = int(num_splits)
     a.stats = _ptr(stats)
+    _decode_cache(a, k, v, k_scale, v_scale)
     _check(lib.mala_decode_noalloc(ctypes.byref(a), _stream(stream)))
     del keep_alive
     return o, lse, keep_mask, int(a.num_splits)
