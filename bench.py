@@ -120,7 +120,6 @@ def _dist_init():
 # are the same at both sizes). Set an entry to None when its kernel changes.
 NCU_TRAFFIC = {
     "mala_bwd_tc_kernel": 8.30e9 + 4.12e9,
-    "mala_decode_split_kernel@131072": (2.148422e9 - 2.147484e9) + 2.147484e9 * 16 + 7.1e6,
 }
 
 

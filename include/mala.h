@@ -232,7 +232,8 @@ typedef struct {
    * for every tensor). An e4m3 cache holds codes whose values are
    * code * k_scale for K and code * v_scale for V (positive, finite; unused
    * for bf16); q stays bf16. The scores then use the query rounded to f16
-   * (exact for |q| >= 2^-14) and P in f16. */
+   * (exact for |q| >= 2^-14) and P in f16. The NaN codes (0x7F, 0xFF) have
+   * no defined result. */
   int32_t kv_dtype;
   float k_scale;
   float v_scale;

@@ -44,9 +44,6 @@
 #include "kernels.h"
 #include "ptx.cuh"
 
-#ifndef MALA_E4M3_CVT
-#define MALA_E4M3_CVT 1       // 0: convert with integer operations and an f16 multiply
-#endif
 #ifndef MALA_DECODE_BF16_WARPS
 #define MALA_DECODE_BF16_WARPS 4
 #endif
@@ -85,26 +82,16 @@ struct Smem {
   static constexpr uint32_t kV = kK + kNSK * kRing;
   static constexpr uint32_t kP = kV + kNSV * kRing;                     // [kNSV][16][kPStride] bf16 / f16
   static constexpr uint32_t kPendM = kP + kNSV * 16 * kPStride * 2;      // [kNSV][16] float
-  static constexpr uint32_t kPMax = kPendM + kNSV * 16 * 4;              // [2][kCW][16] float
-  static constexpr uint32_t kPSum = kPMax + 2 * kCW * 16 * 4;            // [2][kCW][16] float
+  static constexpr uint32_t kPMax = kPendM + kNSV * 16 * 4;              // [2][16][kCW] float
+  static constexpr uint32_t kPSum = kPMax + 2 * kCW * 16 * 4;            // [2][16][kCW] float
   static constexpr uint32_t kBars = kPSum + 2 * kCW * 16 * 4;
   static constexpr uint32_t kMisc = kBars + kNumBars * 8;               // misc words
   static constexpr uint32_t kEnd = kMisc + 64;
   static constexpr uint32_t kAlloc = kEnd + 1024;
 };
 static_assert(Smem<false>::kAlloc <= 232448 && Smem<true>::kAlloc <= 232448, "decode CTA exceeds shared memory");
+static_assert(Smem<false>::kPMax % 16 == 0 && Smem<true>::kPMax % 16 == 0, "per-warp row data read as float4");
 static_assert(Smem<false>::kNSK <= kNSKMax && Smem<true>::kNSK <= kNSKMax, "K ring exceeds its barriers");
-
-// Four e4m3 values (bytes of w) to two f16x2 words: bytes 0, 1 -> lo and
-// 2, 3 -> hi, the lower byte in the lower half.
-__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
-#if MALA_E4M3_CVT
-  lo = e4m3x2_to_f16x2(w & 0xFFFFu);
-  hi = e4m3x2_to_f16x2(w >> 16);
-#else
-  e4m3x4_to_f16x4(w, lo, hi);
-#endif
-}
 
 template <bool FP8>
 __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kernel(const __grid_constant__ DecodeParams p) {
@@ -177,6 +164,8 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
     const int h_hi = has_hi ? p.group_heads[hk][row_hi] : 0;
     const float thr2 = p.log2_tau - log2f(static_cast<float>(p.Nk));   // log2(tau / L_0)
     if (warp == 0 && lane == 0) tma_prefetch_desc(&p.tm_v);
+    // log2(e) times the scale of the raw scores (FP8 caches: the key scale)
+    const float sl2 = FP8 ? kLog2e * p.k_scale : kLog2e;
 
     // query A fragments for the 8 k-steps over d = 128; FP8 caches: k-step
     // kk, fragment column 2tq + e (+ 8) holds d = 32tq + 4kk + e (+ 2)
@@ -215,13 +204,29 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
     int kept_heads = 0;
     const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
 
-    auto fold_sums = [&](int par) {
-      float a = 0.0f, c = 0.0f;
+    // per-warp row values [par][row][warp]: combined with float4 reads
+    auto row_max = [&](const float* base, int par, int row) {
+      const float4* v = reinterpret_cast<const float4*>(base + (par * 16 + row) * kCW);
+      float m = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kCW; ++w) {
-        a += sPSum[(par * kCW + w) * 16 + row_lo];
-        c += sPSum[(par * kCW + w) * 16 + row_hi];
+      for (int w4 = 0; w4 < kCW / 4; ++w4) {
+        const float4 x = v[w4];
+        m = fmaxf(m, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
       }
+      return m;
+    };
+    auto row_sum = [&](const float* base, int par, int row) {
+      const float4* v = reinterpret_cast<const float4*>(base + (par * 16 + row) * kCW);
+      float a = 0.0f;
+#pragma unroll
+      for (int w4 = 0; w4 < kCW / 4; ++w4) {
+        const float4 x = v[w4];
+        a += (x.x + x.y) + (x.z + x.w);
+      }
+      return a;
+    };
+    auto fold_sums = [&](int par) {
+      const float a = row_sum(sPSum, par, row_lo), c = row_sum(sPSum, par, row_hi);
       l_lo += a;
       l_hi += c;
     };
@@ -242,16 +247,14 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
           o[nb][0] *= f_lo; o[nb][1] *= f_lo;
           o[nb][2] *= f_hi; o[nb][3] *= f_hi;
         }
-        const uint32_t* prow_lo = reinterpret_cast<const uint32_t*>(sP + (s * 16 + row_lo) * kPStride);
-        const uint32_t* prow_hi = reinterpret_cast<const uint32_t*>(sP + (s * 16 + row_hi) * kPStride);
         const uint32_t vbase = sVa + s * kRing;
         const int mi = lane >> 3, rr = lane & 7;
+        // A fragments of P: matrices (rows 0-7 | 8-15) x (keys 16kk + [0, 8) | + 8)
+        const uint32_t pa = smem_u32(sP) + ((s * 16 + ((mi & 1) << 3) + rr) * kPStride + 8 * (mi >> 1)) * 2;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t a0 = prow_lo[(16 * kk + 2 * tq) >> 1];
-          const uint32_t a1 = prow_hi[(16 * kk + 2 * tq) >> 1];
-          const uint32_t a2 = prow_lo[(16 * kk + 8 + 2 * tq) >> 1];
-          const uint32_t a3 = prow_hi[(16 * kk + 8 + 2 * tq) >> 1];
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(pa + 32 * kk, a0, a1, a2, a3);
           if constexpr (FP8) {
             // n-block nb, fragment column g is value column kKPW w + kNBW g + nb:
             // bytes [kKPW w + kNBW g, + kNBW) of the rows of keys 16kk + 2tq
@@ -264,11 +267,11 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
               r[x] = kNBW == 4 ? ld_shared_u32(a) : ld_shared_u16(a);
             }
             uint32_t b0[kNBW], b1[kNBW];
-            e4m3x4_to_f16(__byte_perm(r[0], r[1], 0x5140), b0[0], b0[1]);
-            e4m3x4_to_f16(__byte_perm(r[2], r[3], 0x5140), b1[0], b1[1]);
+            e4m3x4_to_f16x4(__byte_perm(r[0], r[1], 0x5140), b0[0], b0[1]);
+            e4m3x4_to_f16x4(__byte_perm(r[2], r[3], 0x5140), b1[0], b1[1]);
             if constexpr (kNBW == 4) {
-              e4m3x4_to_f16(__byte_perm(r[0], r[1], 0x7362), b0[2], b0[3]);
-              e4m3x4_to_f16(__byte_perm(r[2], r[3], 0x7362), b1[2], b1[3]);
+              e4m3x4_to_f16x4(__byte_perm(r[0], r[1], 0x7362), b0[2], b0[3]);
+              e4m3x4_to_f16x4(__byte_perm(r[2], r[3], 0x7362), b1[2], b1[3]);
             }
 #pragma unroll
             for (int nb = 0; nb < kNBW; ++nb) mma_f16_16816(o[nb], a0, a1, a2, a3, b0[nb], b1[nb]);
@@ -316,14 +319,10 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               uint32_t b0, b1;
-              e4m3x4_to_f16(w[kk], b0, b1);
+              e4m3x4_to_f16x4(w[kk], b0, b1);
               mma_f16_16816(sacc[nb], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
             }
           }
-#pragma unroll
-          for (int nb = 0; nb < kNBW; ++nb)
-#pragma unroll
-            for (int x = 0; x < 4; ++x) sacc[nb][x] *= p.k_scale;
         } else {
           const int mi = lane >> 3, rr = lane & 7;
 #pragma unroll
@@ -342,27 +341,31 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
         }
       }
       // keys past the cache end (last tile only) do not exist
+      if (j * kBK + kBK > p.Nk) {
+#pragma unroll
+        for (int nb = 0; nb < kNBW; ++nb)
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+            if (j * kBK + kKPW * warp + 8 * nb + 2 * tq + x >= p.Nk) {
+              sacc[nb][x] = -INFINITY;
+              sacc[nb][2 + x] = -INFINITY;
+            }
+      }
       float mx_lo = -INFINITY, mx_hi = -INFINITY;
 #pragma unroll
       for (int nb = 0; nb < kNBW; ++nb) {
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const int key = j * kBK + kKPW * warp + 8 * nb + 2 * tq + x;
-          if (key >= p.Nk) {
-            sacc[nb][x] = -INFINITY;
-            sacc[nb][2 + x] = -INFINITY;
-          }
-          mx_lo = fmaxf(mx_lo, sacc[nb][x]);
-          mx_hi = fmaxf(mx_hi, sacc[nb][2 + x]);
-        }
+        mx_lo = fmaxf(mx_lo, fmaxf(sacc[nb][0], sacc[nb][1]));
+        mx_hi = fmaxf(mx_hi, fmaxf(sacc[nb][2], sacc[nb][3]));
       }
       mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
       mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
       mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
       mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
       if (tq == 0) {
-        sPMax[((t & 1) * kCW + warp) * 16 + row_lo] = mx_lo;
-        sPMax[((t & 1) * kCW + warp) * 16 + row_hi] = mx_hi;
+        // FP8 caches: the scores so far lack the key scale (> 0, so it
+        // commutes with the maximum); it enters here and in sl2 below
+        sPMax[((t & 1) * 16 + row_lo) * kCW + warp] = FP8 ? mx_lo * p.k_scale : mx_lo;
+        sPMax[((t & 1) * 16 + row_hi) * kCW + warp] = FP8 ? mx_hi * p.k_scale : mx_hi;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kKEmpty + ks]);
@@ -371,12 +374,7 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
 
       // previous tile's sums, this tile's maxima, per-head decisions
       if (prev_any) fold_sums((t - 1) & 1);
-      float tm_lo = -INFINITY, tm_hi = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kCW; ++w) {
-        tm_lo = fmaxf(tm_lo, sPMax[((t & 1) * kCW + w) * 16 + row_lo]);
-        tm_hi = fmaxf(tm_hi, sPMax[((t & 1) * kCW + w) * 16 + row_hi]);
-      }
+      const float tm_lo = row_max(sPMax, t & 1, row_lo), tm_hi = row_max(sPMax, t & 1, row_hi);
       const float tm2_lo = tm_lo * kLog2e, tm2_hi = tm_hi * kLog2e;
       const bool keep_lo = has_lo && (l_lo == 0.0f || tm2_lo - (m2_lo + lg2_approx(l_lo)) >= thr2);
       const bool keep_hi = has_hi && (l_hi == 0.0f || tm2_hi - (m2_hi + lg2_approx(l_hi)) >= thr2);
@@ -409,10 +407,10 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
       uint32_t pk_lo[kNBW], pk_hi[kNBW];
 #pragma unroll
       for (int nb = 0; nb < kNBW; ++nb) {
-        const float a0 = keep_lo ? ex2_approx(fmaf(sacc[nb][0], kLog2e, -m2_lo)) : 0.0f;
-        const float a1 = keep_lo ? ex2_approx(fmaf(sacc[nb][1], kLog2e, -m2_lo)) : 0.0f;
-        const float c0 = keep_hi ? ex2_approx(fmaf(sacc[nb][2], kLog2e, -m2_hi)) : 0.0f;
-        const float c1 = keep_hi ? ex2_approx(fmaf(sacc[nb][3], kLog2e, -m2_hi)) : 0.0f;
+        const float a0 = keep_lo ? ex2_approx(fmaf(sacc[nb][0], sl2, -m2_lo)) : 0.0f;
+        const float a1 = keep_lo ? ex2_approx(fmaf(sacc[nb][1], sl2, -m2_lo)) : 0.0f;
+        const float c0 = keep_hi ? ex2_approx(fmaf(sacc[nb][2], sl2, -m2_hi)) : 0.0f;
+        const float c1 = keep_hi ? ex2_approx(fmaf(sacc[nb][3], sl2, -m2_hi)) : 0.0f;
         ps_lo += a0 + a1;
         ps_hi += c0 + c1;
         pk_lo[nb] = FP8 ? pack_f16x2(a0, a1) : pack_bf16x2(a0, a1);
@@ -423,8 +421,8 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
       ps_hi += __shfl_xor_sync(0xffffffffu, ps_hi, 1);
       ps_hi += __shfl_xor_sync(0xffffffffu, ps_hi, 2);
       if (tq == 0) {
-        sPSum[((t & 1) * kCW + warp) * 16 + row_lo] = ps_lo;
-        sPSum[((t & 1) * kCW + warp) * 16 + row_hi] = ps_hi;
+        sPSum[((t & 1) * 16 + row_lo) * kCW + warp] = ps_lo;
+        sPSum[((t & 1) * 16 + row_hi) * kCW + warp] = ps_hi;
       }
       // a free P/V slot: run the oldest pending PV when both are taken
       if (kc - pv_done == kNSV) do_pv();

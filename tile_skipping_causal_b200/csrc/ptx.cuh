@@ -349,30 +349,14 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
   return pack_f16x2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
-// Two e4m3 values (byte 0 -> low half, byte 1 -> high half) to f16x2; every
-// e4m3 value is exactly representable in f16.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
-  uint32_t r;
-  asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(r) : "r"(two_bytes));
-  return r;
-}
-
-// Four e4m3 values (bytes 0..3 of w) to two f16x2 words (bytes 0, 1 -> lo;
-// 2, 3 -> hi) with integer operations and one f16 multiply: each byte's
-// exponent and mantissa bits are placed at the f16 exponent / mantissa
-// positions (bits 13..7), which reads as 2^-8 times the e4m3 value (its bias
-// 7 against f16's 15; subnormals map to f16 subnormals), with the sign at
-// bit 15; the multiply by 2^8 is then exact.
+// Four e4m3 values (bytes 0..3 of w) to two f16x2 words: bytes 0, 1 -> lo,
+// bytes 2, 3 -> hi, the lower byte in the lower half. Every e4m3 value is
+// exactly representable in f16.
 __device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const uint32_t a = __byte_perm(w, 0u, 0x4140);   // [0, b1, 0, b0]
-  const uint32_t c = __byte_perm(w, 0u, 0x4342);   // [0, b3, 0, b2]
-  const uint32_t a16 = ((a << 7) & 0x3F803F80u) | ((a << 8) & 0x80008000u);
-  const uint32_t c16 = ((c << 7) & 0x3F803F80u) | ((c << 8) & 0x80008000u);
-  const __half2 k256 = __half2(__ushort_as_half(0x5C00), __ushort_as_half(0x5C00));
-  __half2 x = __hmul2(*reinterpret_cast<const __half2*>(&a16), k256);
-  __half2 y = __hmul2(*reinterpret_cast<const __half2*>(&c16), k256);
-  lo = *reinterpret_cast<uint32_t*>(&x);
-  hi = *reinterpret_cast<uint32_t*>(&y);
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
 __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
