@@ -120,6 +120,10 @@ def _dist_init():
 # are the same at both sizes). Set an entry to None when its kernel changes.
 NCU_TRAFFIC = {
     "mala_bwd_tc_kernel": 8.30e9 + 4.12e9,
+    # decode at N_k = 8192 (ncu): reads beyond the K/V cache + the cache x 16
+    # (N_k = 131072) + writes (outputs and split partials, independent of N_k)
+    "mala_decode_split_kernel@131072": (2.148081e9 - 2.147484e9) + 2.147484e9 * 16 + 7.04e6,
+    "mala_decode_split_kernel@131072/e4m3": (1.077085e9 - 1.073742e9) + 1.073742e9 * 16 + 8.57e6,
 }
 
 
@@ -496,7 +500,7 @@ def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072, e4m3: bool = 
             "roofline": {"bound": "hbm", "kernel": "mala_decode_split_kernel", "achieved": gbs,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                          "peak_source": f"{peaks['source']} hbm_gbs",
-                         "traffic": None if e4m3 else NCU_TRAFFIC.get(f"mala_decode_split_kernel@{w.seqlen_k}"),
+                         "traffic": NCU_TRAFFIC.get(f"mala_decode_split_kernel@{w.seqlen_k}" + ("/e4m3" if e4m3 else "")),
                          "traffic_note": "ncu DRAM bytes per launch, N_k = 8192 capture scaled by N_k"}}
 
 
