@@ -35,6 +35,10 @@ extracted, so each test is restated from the surrounding prose:
 * decode: L_0 = N_k (the current token included); split p covers key tiles
   [floor(p T / P), floor((p+1) T / P)) of the T tiles, visited descending,
   with its own (m, l); partial outputs merge by their log-normalizers.
+* group-joint decode (the pages only say that every valid row of a query
+  block must pass for a tile to be skipped): the query heads of a GQA group
+  are taken as the rows of one block, so the group takes one decision per
+  key tile and every head accumulates the retained tiles.
 
 Readings taken where the page is silent (each also listed in the design
 notes): skip is the strict "<" so a tie retains; tau = 0 means log tau = -inf
@@ -357,6 +361,45 @@ def decode_head(q_row: np.ndarray, K: np.ndarray, V: np.ndarray, B_k: int,
             margin[j] = st["margin"][j]
     O, z = merge_partials(partials)
     return O, z, keep, margin, partials
+
+
+def decode_group(Q_rows: np.ndarray, K: np.ndarray, V: np.ndarray, B_k: int,
+                 tau: float, num_splits: int = 1, replay=None):
+    """Group-joint decoding: the G query heads that share one KV head take one
+    decision per key tile. The heads' query rows (each at position N_k - 1,
+    L_0 = N_k) are treated like the rows of one query block under the test of
+    "Online Sparse Softmax": a tile is skipped only when every head passes the
+    skip test, and a retained tile updates every head. Splits as in
+    ``decode_head``, each with its own (m, l) per head.
+
+    replay: optional bool [nKB] forcing the per-tile decisions.
+    Returns O [G, d], z [G], keep [nKB] bool, margin [nKB]."""
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    Qg = np.asarray(Q_rows, dtype=np.float64)
+    G = Qg.shape[0]
+    N_k = K.shape[0]
+    nKB = num_blocks(N_k, B_k)
+    pos = np.full(G, N_k - 1)
+    L = np.full(G, N_k)
+    keep = np.zeros(nKB, dtype=bool)
+    margin = np.full(nKB, np.nan)
+    partials = [[] for _ in range(G)]
+    for (t0, t1) in split_ranges(nKB, num_splits):
+        tiles = list(range(t1 - 1, t0 - 1, -1))
+        rep = None if replay is None else {j: bool(replay[j]) for j in tiles}
+        st = forward_block(Qg, pos, K, V, B_k, tau, tiles, L_i=L, replay=rep)
+        O_p, z_p = finalize(st)
+        for g in range(G):
+            partials[g].append((O_p[g], float(z_p[g])))
+        for j in tiles:
+            keep[j] = st["keep"][j]
+            margin[j] = st["margin"][j]
+    O = np.zeros((G, V.shape[1]))
+    z = np.zeros(G)
+    for g in range(G):
+        O[g], z[g] = merge_partials(partials[g])
+    return O, z, keep, margin
 
 
 def merge_partials(partials):

@@ -405,6 +405,101 @@ def test_decode_first_tile_of_each_split_retained():
     assert orc.split_ranges(10, 3) == [(0, 3), (3, 6), (6, 10)]
 
 
+def _group_case(seed, G, N, d, sharp=3.0):
+    rng = np.random.default_rng(seed)
+    Qg = rng.standard_normal((G, d)) * sharp / math.sqrt(d)
+    K = rng.standard_normal((N, d))
+    V = rng.standard_normal((N, d))
+    return Qg, K, V
+
+
+@pytest.mark.parametrize("P", [1, 3])
+def test_decode_group_of_one_is_per_head_decode(P):
+    Qg, K, V = _group_case(50 + P, 1, 77, 6)
+    for tau in (0.05, 0.5, 4.0):
+        O, z, keep, margin = orc.decode_group(Qg, K, V, 8, tau, P)
+        Oh, zh, kh, mh, _ = orc.decode_head(Qg[0], K, V, 8, tau, P)
+        assert (keep == kh).all()
+        assert np.allclose(O[0], Oh, atol=1e-14) and abs(z[0] - zh) < 1e-14
+
+
+def test_decode_group_of_identical_heads_is_per_head_decode():
+    Qg, K, V = _group_case(60, 1, 90, 5)
+    Qg = np.repeat(Qg, 4, axis=0)
+    O, z, keep, _ = orc.decode_group(Qg, K, V, 8, 0.5, 2)
+    Oh, zh, kh, _, _ = orc.decode_head(Qg[0], K, V, 8, 0.5, 2)
+    assert (keep == kh).all()
+    for g in range(4):
+        assert np.allclose(O[g], Oh, atol=1e-14) and abs(z[g] - zh) < 1e-14
+
+
+@pytest.mark.parametrize("P", [1, 2, 5])
+def test_decode_group_at_tau_zero_is_dense(P):
+    Qg, K, V = _group_case(70 + P, 4, 61, 5)
+    O, z, keep, _ = orc.decode_group(Qg, K, V, 8, 0.0, P)
+    assert keep.all()
+    for g in range(4):
+        s = K @ Qg[g]
+        w = np.exp(s - s.max())
+        assert np.allclose(O[g], (w / w.sum()) @ V, atol=1e-13)
+        assert abs(z[g] - (s.max() + math.log(w.sum()))) < 1e-13
+
+
+@pytest.mark.parametrize("seed,P,tau", [(80, 1, 0.3), (81, 2, 1.0), (82, 3, 3.0), (83, 1, 20.0)])
+def test_decode_group_brute_force(seed, P, tau):
+    """The joint decisions re-derived from their definition, in ratio form with
+    explicit retained key sets: within a split, walking its tiles from the
+    last, a tile is retained iff the retained set is still empty or some head
+    has a key in the tile with exp(s) / sum over retained keys of exp(s) >=
+    tau / N_k. Every head's output is then plain softmax attention over the
+    keys of all retained tiles."""
+    G, N, d, Bk = 4, 70, 4, 8
+    Qg, K, V = _group_case(seed, G, N, d, sharp=6.0)
+    O, z, keep, _ = orc.decode_group(Qg, K, V, Bk, tau, P)
+    S = Qg @ K.T                                     # [G, N]
+    nKB = -(-N // Bk)
+    want = np.zeros(nKB, dtype=bool)
+    for (t0, t1) in orc.split_ranges(nKB, P):
+        kept_keys = []
+        for j in range(t1 - 1, t0 - 1, -1):
+            keys = list(range(j * Bk, min((j + 1) * Bk, N)))
+            if not kept_keys:
+                want[j] = True
+            else:
+                mass = np.exp(S[:, kept_keys]).sum(axis=1)          # [G]
+                ratio = np.exp(S[:, keys]).max(axis=1) / mass
+                want[j] = bool((ratio >= tau / N).any())
+            if want[j]:
+                kept_keys += keys
+    assert (keep == want).all()
+    if tau >= 3.0:
+        assert keep.sum() < nKB                      # the case does skip
+    cols = np.concatenate([np.arange(j * Bk, min((j + 1) * Bk, N)) for j in range(nKB) if want[j]])
+    for g in range(G):
+        w = np.exp(S[g, cols])
+        assert np.allclose(O[g], (w / w.sum()) @ V[cols], atol=1e-12)
+        assert abs(z[g] - math.log(w.sum())) < 1e-12
+
+
+def test_decode_group_retains_a_tile_one_head_needs():
+    """A tile that only one head of the group needs is retained for all heads;
+    per-head decode would read it for that head alone."""
+    G, N, d, Bk = 3, 64, 4, 8
+    rng = np.random.default_rng(90)
+    K = rng.standard_normal((N, d)) * 0.1
+    V = rng.standard_normal((N, d))
+    Qg = np.zeros((G, d))
+    Qg[:, 0] = 1.0
+    K[5, 1] = 40.0                                   # a key only head 2 scores highly
+    Qg[2, 1] = 1.0
+    O, z, keep, _ = orc.decode_group(Qg, K, V, Bk, 2.0, 1)
+    _, z0, k0, _, _ = orc.decode_head(Qg[0], K, V, Bk, 2.0, 1)
+    _, _, k2, _, _ = orc.decode_head(Qg[2], K, V, Bk, 2.0, 1)
+    assert k2[0] and not k0[0] and keep[0]
+    assert (keep >= k0).all()
+    assert z[0] > z0                                 # head 0 now also holds tile 0's mass
+
+
 def test_replay_forces_decisions_but_keeps_margins():
     Q, K, V = _rand_case(41, 32, 4, sharp=5.0)
     O, z, keep, margin = orc.forward_head(Q, K, V, 8, 8, 0.5)
