@@ -483,6 +483,27 @@ def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072, e4m3: bool = 
     torch.cuda.synchronize()
     mala.check_device_error()
     t = e0.elapsed_time(e1) / 1e3 / n
+    group = None
+    if not e4m3:
+        # group-joint voting (one decision per key tile for the query heads of
+        # a KV head) on the same cache
+        gstats = torch.zeros(4, dtype=torch.int64, device=dev)
+        mala.mala_decode(q, k, v, w.tau, 128, P, o=out, lse=l2, keep_mask=km, workspace=workspace,
+                         stats=gstats, group_vote=True)
+        for _ in range(3):
+            mala.mala_decode(q, k, v, w.tau, 128, P, o=out, lse=l2, keep_mask=km, workspace=workspace,
+                             group_vote=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n):
+            mala.mala_decode(q, k, v, w.tau, 128, P, o=out, lse=l2, keep_mask=km, workspace=workspace,
+                             group_vote=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        mala.check_device_error()
+        tg = e0.elapsed_time(e1) / 1e3 / n
+        gt, gv = (int(x) for x in gstats.cpu().tolist()[:2])
+        group = {"ms": tg * 1e3, "tokens_per_s": w.batch / tg, "v_tiles_read": gv, "v_read_fraction": gv / gt}
     d = w.head_dim
     kbytes = w.batch * w.heads_kv * w.seqlen_k * d * esz
     vbytes = vread * 128 * d * esz
@@ -501,7 +522,8 @@ def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072, e4m3: bool = 
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                          "peak_source": f"{peaks['source']} hbm_gbs",
                          "traffic": NCU_TRAFFIC.get(f"mala_decode_split_kernel@{w.seqlen_k}" + ("/e4m3" if e4m3 else "")),
-                         "traffic_note": "ncu DRAM bytes per launch, N_k = 8192 capture scaled by N_k"}}
+                         "traffic_note": "ncu DRAM bytes per launch, N_k = 8192 capture scaled by N_k"},
+            "group_vote": group}
 
 
 _ORACLE_INPUTS = {}

@@ -237,6 +237,14 @@ typedef struct {
   int32_t kv_dtype;
   float k_scale;
   float v_scale;
+  /* 0 (the default): every query head decides for itself ("Online Sparse
+   * Softmax" applied per head). 1: group-joint voting, one decision per key
+   * tile for all query heads that share a KV head: their rows are treated
+   * like the rows of one query block, so a tile is skipped only when every
+   * head of the group passes the skip test, and a retained tile is
+   * accumulated by every head of the group. keep_mask bits are then equal
+   * across a group. Other values: MALA_ERR_INVALID_ARG. */
+  int32_t group_vote;
 } mala_decode_args;
 
 MALA_API size_t mala_decode_workspace_size(const mala_decode_args* args);

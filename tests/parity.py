@@ -169,6 +169,48 @@ def check_decode(q, k, v, o, lse, keep_words, tau, P, B_k=128, heads=None, rep=N
     return rep
 
 
+def check_decode_group(q, k, v, o, lse, keep_words, tau, P, B_k=128, groups=None, rep=None):
+    """mala_decode(group_vote=True) vs the oracle's group-joint decoding for
+    (batch, KV head) pairs ``groups`` (None = all), default head map. The
+    heads of a group must carry identical keep bits; a decision that differs
+    from the oracle's must lie inside the margin band (the oracle then
+    replays the GPU's decisions); every head's O and LSE must match."""
+    rep = rep or DecReport()
+    B, _, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    nKB = orc.num_blocks(Nk, B_k)
+    keep = mala.unpack_mask(keep_words, nKB)
+    if groups is None:
+        groups = [(b, hk) for b in range(B) for hk in range(Hkv)]
+    o_c = f64(o)
+    lse_c = lse.detach().cpu().numpy()
+    for (b, hk) in groups:
+        h0 = hk * G
+        gk = np.asarray(keep[b, h0, :nKB], dtype=bool)
+        for h in range(h0 + 1, h0 + G):
+            assert (np.asarray(keep[b, h, :nKB], dtype=bool) == gk).all(), \
+                f"group b={b} hk={hk}: heads {h0} and {h} carry different keep bits"
+        Qg = f64(q[b, 0, h0:h0 + G])
+        K, V = f64(k[b, :, hk]), f64(v[b, :, hk])
+        O, z, okeep, margin = orc.decode_group(Qg, K, V, B_k, tau, P)
+        if (okeep != gk).any():
+            rep.replayed += 1
+            O, z, okeep, margin = orc.decode_group(Qg, K, V, B_k, tau, P, replay=gk)
+        for j in range(nKB):
+            if gk[j] != (margin[j] <= 0.0):
+                assert abs(margin[j]) <= MARGIN_BAND, \
+                    f"group b={b} hk={hk}: tile {j} decided {gk[j]} with margin {margin[j]:.3e}"
+                rep.band_flips += 1
+        for i in range(G):
+            assert_close(o_c[b, 0, h0 + i], O[i], f"group decode b={b} h={h0 + i} O")
+            assert_close(np.array([lse_c[b, h0 + i]]), np.array([z[i]]), f"group decode b={b} h={h0 + i} LSE")
+            rep.heads += 1
+        rep.tiles += nKB
+        rep.kept += int(gk.sum())
+    return rep
+
+
 def oracle_forward_replaying(q64, k64, v64, b, h, G, blocks, gpu_keep_bh, B_q, B_k, tau, rep=None):
     """Oracle O and z for query blocks ``blocks`` of head (b, h), with the
     GPU's forward decisions forced; every forced decision that differs from

@@ -201,3 +201,30 @@ def test_backward_checks_packed_offsets_too(lib):
     arr_k, a.cu_seqlens_k = _cu(0, 100, 256)         # the first sequence has more queries than keys
     assert lib.mala_bwd_workspace_size(ctypes.byref(a)) == 0
     assert lib.mala_bwd(ctypes.byref(a), None, 0, None) == mala.MALA_ERR_UNSUPPORTED
+
+
+def _decode_args(**kw):
+    a = mala.DecodeArgs()
+    fake = 0x10000
+    a.q = a.k = a.v = a.o = a.lse = fake
+    a.batch, a.heads_q, a.heads_kv, a.seqlen_k, a.head_dim = 2, 8, 2, 1000, 128
+    for s in ("q_stride", "o_stride"):
+        setattr(a, s, mala._i64x3(8 * 128, 8 * 128, 128))
+    for s in ("k_stride", "v_stride"):
+        setattr(a, s, mala._i64x3(1000 * 2 * 128, 2 * 128, 128))
+    a.block_k = 128
+    a.tau = 0.1
+    a.dtype = mala.MALA_BF16
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw", [dict(group_vote=2), dict(group_vote=-1), dict(kv_dtype=5),
+                                dict(kv_dtype=mala.MALA_FP8_E4M3, k_scale=0.0, v_scale=1.0),
+                                dict(num_splits=9)])
+def test_decode_rejects_bad_arguments_without_launching(lib, kw):
+    a = _decode_args(**kw)
+    assert lib.mala_decode_workspace_size(ctypes.byref(a)) == 0
+    assert lib.mala_decode(ctypes.byref(a), None, 0, None) == mala.MALA_ERR_INVALID_ARG
+    assert lib.mala_last_error_message().decode()

@@ -7,7 +7,7 @@ import torch
 
 from oracle import mala_oracle as orc
 from tile_skipping_causal_b200 import mala, synth
-from tests.parity import check_decode
+from tests.parity import check_decode, check_decode_group
 
 pytestmark = pytest.mark.gpu
 
@@ -167,3 +167,38 @@ def test_decode_e4m3_rejects_bad_scales():
         mala.mala_decode(q, kc, vc, w.tau, k_scale=0.0)
     with pytest.raises(ValueError):
         mala.mala_decode(q, kc, v, w.tau)            # mixed cache types
+
+
+# ------------------------------------------------------ group-joint voting
+
+@pytest.mark.parametrize("Nk,splits,tau", [(1000, 1, 0.05), (1000, 3, 5.0), (4096, 0, 5.0),
+                                           (4096, 1, 50.0), (129, 0, 50.0)])
+def test_decode_group_vote_matches_oracle(Nk, splits, tau):
+    w, q, k, v = _small(2, Nk, seed=11)
+    stats = torch.zeros(4, dtype=torch.int64, device=DEV)
+    o, lse, keep, P = _decode(q, k, v, tau, splits, group_vote=True, stats=stats)
+    rep = check_decode_group(q, k, v, o, lse, keep, tau, P)
+    assert rep.heads == 2 * 32
+    tested, vread, kept_heads = (int(x) for x in stats.cpu().tolist()[:3])
+    assert tested == 2 * 8 * -(-Nk // 128)
+    assert kept_heads == 4 * vread                   # every head accumulates every V tile read
+    if tau >= 50.0 and Nk > 1000:
+        assert vread < tested                        # the case does skip
+
+
+def test_decode_group_vote_with_single_head_groups_is_per_head():
+    w, q, k, v = _small(2, 2000, seed=12, Hq=8, Hkv=8)
+    a = _decode(q, k, v, 5.0, 0)
+    b = _decode(q, k, v, 5.0, 0, group_vote=True)
+    assert a[3] == b[3]
+    for x, y in zip(a[:3], b[:3]):
+        assert torch.equal(x, y)
+
+
+def test_decode_group_vote_e4m3_cache():
+    w, q, k, v = _small(1, 3000, seed=13)
+    kc, kd = _quantise(k, 0.5)
+    vc, vd = _quantise(v, 1.0)
+    o, lse, keep, P = _decode(q, kc, vc, 5.0, 0, group_vote=True, k_scale=0.5, v_scale=1.0)
+    rep = check_decode_group(q, kd, vd, o, lse, keep, 5.0, P)
+    assert rep.heads == 32

@@ -376,9 +376,15 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
       if (prev_any) fold_sums((t - 1) & 1);
       const float tm_lo = row_max(sPMax, t & 1, row_lo), tm_hi = row_max(sPMax, t & 1, row_hi);
       const float tm2_lo = tm_lo * kLog2e, tm2_hi = tm_hi * kLog2e;
-      const bool keep_lo = has_lo && (l_lo == 0.0f || tm2_lo - (m2_lo + lg2_approx(l_lo)) >= thr2);
-      const bool keep_hi = has_hi && (l_hi == 0.0f || tm2_hi - (m2_hi + lg2_approx(l_hi)) >= thr2);
-      const bool any = __any_sync(0xffffffffu, keep_lo || keep_hi);
+      bool keep_lo = has_lo && (l_lo == 0.0f || tm2_lo - (m2_lo + lg2_approx(l_lo)) >= thr2);
+      bool keep_hi = has_hi && (l_hi == 0.0f || tm2_hi - (m2_hi + lg2_approx(l_hi)) >= thr2);
+      const bool any = __any_sync(0xffffffffu, keep_lo || keep_hi);   // over all 16 rows
+      if (p.group_vote) {
+        // group-joint voting: the group's rows decide together, like the
+        // rows of one query block; every head accumulates a retained tile
+        keep_lo = has_lo && any;
+        keep_hi = has_hi && any;
+      }
       if (warp == 0 && tq == 0) {
         if (keep_lo) { mw_lo |= 1u << (j & 31); ++kept_heads; }
         if (keep_hi) { mw_hi |= 1u << (j & 31); ++kept_heads; }

@@ -85,6 +85,7 @@ struct DecodeParams {
   float log2_tau;
   int kv_fp8;           // K and V cache in e4m3 (tm_k / tm_v are then byte maps)
   float k_scale, v_scale;   // e4m3 cache scales (value = code * scale)
+  int group_vote;       // one decision per key tile for the whole query-head group
   uint8_t group_size[kMaxKvHeads];
   uint8_t group_heads[kMaxKvHeads][kMaxGroup];
 };

@@ -500,6 +500,8 @@ int decode_check(const mala_decode_args* a, int* nKB_out) {
   if (a->kv_dtype != MALA_BF16 && a->kv_dtype != MALA_FP8_E4M3)
     return fail(MALA_ERR_INVALID_ARG, "kv_dtype %d is neither MALA_BF16 nor MALA_FP8_E4M3", a->kv_dtype);
   const bool fp8 = a->kv_dtype == MALA_FP8_E4M3;
+  if (a->group_vote != 0 && a->group_vote != 1)
+    return fail(MALA_ERR_INVALID_ARG, "group_vote %d is neither 0 nor 1", a->group_vote);
   if (fp8 && !(a->k_scale > 0.0f && a->k_scale < INFINITY && a->v_scale > 0.0f && a->v_scale < INFINITY))
     return fail(MALA_ERR_INVALID_ARG, "e4m3 cache scales must be positive and finite");
   const int64_t kes = fp8 ? 1 : 2;
@@ -583,6 +585,7 @@ int mala_decode(mala_decode_args* a, void* workspace, size_t ws_bytes, void* str
     p.group_heads[hk][p.group_size[hk]++] = static_cast<uint8_t>(h);
   }
   if ((rc = decode_cache_maps(a, &p))) return rc;
+  p.group_vote = a->group_vote;
   p.err = device_error_ptr();
   if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
   p.q = a->q;
@@ -684,6 +687,7 @@ extern "C" int mala_decode_noalloc(mala_decode_args* a, void* stream_) {
     p.group_heads[hk][p.group_size[hk]++] = static_cast<uint8_t>(h);
   }
   if ((rc = decode_cache_maps(a, &p))) return rc;
+  p.group_vote = a->group_vote;
   p.err = device_error_ptr();
   if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
   p.q = a->q;

@@ -65,6 +65,7 @@ class DecodeArgs(ctypes.Structure):
         ("q_to_kv", ctypes.c_void_p), ("block_k", ctypes.c_int32), ("tau", ctypes.c_float),
         ("dtype", ctypes.c_int32), ("num_splits", ctypes.c_int32), ("stats", ctypes.c_void_p),
         ("kv_dtype", ctypes.c_int32), ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
+        ("group_vote", ctypes.c_int32),
     ]
 
 
@@ -337,11 +338,14 @@ def _decode_cache(a, k, v, k_scale, v_scale):
 
 def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *, o=None,
                 lse=None, keep_mask=None, with_mask: bool = True, stats=None, q_to_kv=None,
-                stream=None, workspace=None, k_scale: float = 1.0, v_scale: float = 1.0):
+                stream=None, workspace=None, k_scale: float = 1.0, v_scale: float = 1.0,
+                group_vote: bool = False):
     """Single-token decoding. q [B, 1, Hq, d] bf16; k/v cache [B, Nk, Hkv, d]
     in bf16, or torch.float8_e4m3fn codes whose values are code * k_scale and
-    code * v_scale. Returns (o, lse [B, Hq], keep_mask words
-    [B, Hq, ceil(T/32)] or None, num_splits used)."""
+    code * v_scale. group_vote: one decision per key tile for all query heads
+    of a KV head (a tile is skipped only when every head passes the test).
+    Returns (o, lse [B, Hq], keep_mask words [B, Hq, ceil(T/32)] or None,
+    num_splits used)."""
     lib = load_library()
     _require_cuda(q, k, v)
     B, _, Hq, d = q.shape
@@ -364,6 +368,7 @@ def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *,
     a.num_splits = int(num_splits)
     a.stats = _ptr(stats)
     _decode_cache(a, k, v, k_scale, v_scale)
+    a.group_vote = 1 if group_vote else 0
     ws_n = lib.mala_decode_workspace_size(ctypes.byref(a))
     own_ws = workspace is None or workspace.numel() < ws_n
     if own_ws:
@@ -377,7 +382,8 @@ def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *,
 
 def mala_decode_noalloc(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *, o=None,
                         lse=None, keep_mask=None, with_mask: bool = True, stats=None, q_to_kv=None,
-                        stream=None, k_scale: float = 1.0, v_scale: float = 1.0):
+                        stream=None, k_scale: float = 1.0, v_scale: float = 1.0,
+                        group_vote: bool = False):
     """mala_decode without a workspace: the library keeps the split partials
     in its own built-in device buffer (for callers that cannot allocate;
     calls that overlap on the GPU race on that buffer). Returns the same
@@ -404,6 +410,7 @@ def mala_decode_noalloc(q, k, v, tau: float, block_k: int = 128, num_splits: int
     a.num_splits = int(num_splits)
     a.stats = _ptr(stats)
     _decode_cache(a, k, v, k_scale, v_scale)
+    a.group_vote = 1 if group_vote else 0
     _check(lib.mala_decode_noalloc(ctypes.byref(a), _stream(stream)))
     del keep_alive
     return o, lse, keep_mask, int(a.num_splits)
