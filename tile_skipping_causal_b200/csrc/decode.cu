@@ -56,7 +56,7 @@ constexpr int kBK = 128;
 constexpr int kD = 128;
 constexpr int kNSKMax = 8;              // K ring stages: 4 bf16 tiles, 8 e4m3 tiles
 constexpr int kNSV = 2;                 // V / P slots
-constexpr uint32_t kTileBytes = kBK * kD * 2;   // bf16 tile (and staging tile)
+constexpr uint32_t kTileBytes = kBK * kD * 2;   // bf16 tile
 constexpr int kPStride = 136;           // bf16 per P row (128 + 8 padding)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
