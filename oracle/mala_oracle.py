@@ -35,10 +35,11 @@ extracted, so each test is restated from the surrounding prose:
 * decode: L_0 = N_k (the current token included); split p covers key tiles
   [floor(p T / P), floor((p+1) T / P)) of the T tiles, visited descending,
   with its own (m, l); partial outputs merge by their log-normalizers.
-* group-joint decode (the pages only say that every valid row of a query
-  block must pass for a tile to be skipped): the query heads of a GQA group
-  are taken as the rows of one block, so the group takes one decision per
-  key tile and every head accumulates the retained tiles.
+* group-joint decode and prefill (the pages only say that every valid row
+  of a query block must pass for a tile to be skipped): the query heads of a
+  GQA group are taken as the rows of one block (decode: the heads' single
+  rows; prefill: the heads' rows of the same query block), so the group
+  takes one decision per tile and every head accumulates the retained tiles.
 
 Readings taken where the page is silent (each also listed in the design
 notes): skip is the strict "<" so a tie retains; tau = 0 means log tau = -inf
@@ -194,6 +195,47 @@ def forward_head(Q: np.ndarray, K: np.ndarray, V: np.ndarray, B_q: int,
             rep = {j: bool(replay_mask[i, j]) for j in tiles}
         st = forward_block(Q[q0:q1], pos, K, V, B_k, tau, tiles, replay=rep)
         O[q0:q1], z[q0:q1] = finalize(st)
+        for j in tiles:
+            keep[i, j] = st["keep"][j]
+            margin[i, j] = st["margin"][j]
+    return O, z, keep, margin
+
+
+def forward_group(Qg: np.ndarray, K: np.ndarray, V: np.ndarray, B_q: int,
+                  B_k: int, tau: float, replay_mask: Optional[np.ndarray] = None,
+                  blocks: Optional[Iterable[int]] = None):
+    """Group-joint prefill: the G query heads that share one KV head take one
+    decision per (query block, key tile). For query block i the G heads'
+    rows are taken together as the rows of one block under the test of
+    "Online Sparse Softmax" (skipped only when every row of every head
+    passes; a retained tile updates every head). Causal, N_q <= N_k,
+    bottom-right aligned as in ``forward_head``.
+
+    Qg [G, N_q, d]. Returns O [G, N_q, d], z [G, N_q], keep [nQB, nKB] bool,
+    margin [nQB, nKB] (NaN where a tile is never visited)."""
+    Qg = np.asarray(Qg, dtype=np.float64)
+    G, N_q, d = Qg.shape
+    N_k = K.shape[0]
+    assert N_q <= N_k, "causal mode needs N_q <= N_k (bottom-right alignment)"
+    off = N_k - N_q
+    nQB, nKB = num_blocks(N_q, B_q), num_blocks(N_k, B_k)
+    O = np.full((G, N_q, V.shape[1]), np.nan)
+    z = np.full((G, N_q), np.nan)
+    keep = np.zeros((nQB, nKB), dtype=bool)
+    margin = np.full((nQB, nKB), np.nan)
+    for i in (range(nQB) if blocks is None else blocks):
+        q0, q1 = i * B_q, min((i + 1) * B_q, N_q)
+        R = q1 - q0
+        rows = Qg[:, q0:q1].reshape(G * R, d)            # head-major stack of the block's rows
+        pos = np.tile(np.arange(q0, q1) + off, G)
+        tiles = causal_tiles(q1 - 1 + off, B_k, nKB)
+        rep = None
+        if replay_mask is not None:
+            rep = {j: bool(replay_mask[i, j]) for j in tiles}
+        st = forward_block(rows, pos, K, V, B_k, tau, tiles, replay=rep)
+        Ob, zb = finalize(st)
+        O[:, q0:q1] = Ob.reshape(G, R, -1)
+        z[:, q0:q1] = zb.reshape(G, R)
         for j in tiles:
             keep[i, j] = st["keep"][j]
             margin[i, j] = st["margin"][j]

@@ -500,6 +500,96 @@ def test_decode_group_retains_a_tile_one_head_needs():
     assert z[0] > z0                                 # head 0 now also holds tile 0's mass
 
 
+@pytest.mark.parametrize("Nq,Nk", [(40, 40), (29, 45)])
+def test_forward_group_of_one_is_forward_head(Nq, Nk):
+    rng = np.random.default_rng(100 + Nq)
+    Q = rng.standard_normal((1, Nq, 5)) * 4 / math.sqrt(5)
+    K = rng.standard_normal((Nk, 5))
+    V = rng.standard_normal((Nk, 5))
+    for tau in (0.1, 1.0, 10.0):
+        O, z, keep, margin = orc.forward_group(Q, K, V, 8, 8, tau)
+        Oh, zh, kh, mh = orc.forward_head(Q[0], K, V, 8, 8, tau)
+        assert (keep == kh).all()
+        assert np.allclose(O[0], Oh, atol=1e-14) and np.allclose(z[0], zh, atol=1e-14)
+
+
+def test_forward_group_of_identical_heads_is_forward_head():
+    rng = np.random.default_rng(110)
+    Q1 = rng.standard_normal((37, 4)) * 4 / 2
+    K = rng.standard_normal((37, 4))
+    V = rng.standard_normal((37, 4))
+    O, z, keep, _ = orc.forward_group(np.stack([Q1] * 3), K, V, 8, 8, 1.0)
+    Oh, zh, kh, _ = orc.forward_head(Q1, K, V, 8, 8, 1.0)
+    assert (keep == kh).all()
+    for g in range(3):
+        assert np.allclose(O[g], Oh, atol=1e-14) and np.allclose(z[g], zh, atol=1e-14)
+
+
+def test_forward_group_at_tau_zero_is_dense():
+    rng = np.random.default_rng(120)
+    G, N, d = 3, 33, 4
+    Qg = rng.standard_normal((G, N, d)) * 2
+    K = rng.standard_normal((N, d))
+    V = rng.standard_normal((N, d))
+    O, z, keep, _ = orc.forward_group(Qg, K, V, 8, 8, 0.0)
+    for g in range(G):
+        _, _, _, Od, zd, _ = _dense_torch(Qg[g], K, V)
+        assert np.allclose(O[g], Od.detach().numpy(), atol=1e-12)
+        assert np.allclose(z[g], zd.detach().numpy(), atol=1e-12)
+
+
+@pytest.mark.parametrize("seed,tau,Nq", [(130, 0.5, 48), (131, 300.0, 48), (132, 300.0, 41)])
+def test_forward_group_brute_force(seed, tau, Nq):
+    """Joint decisions from their definition in ratio form, with explicit
+    retained key sets per row: a tile is retained iff some row of some head
+    with a legal key in it has an empty retained set or a key whose
+    exp(s) / sum over its retained keys of exp(s) is >= tau / L_q; every row's
+    output is softmax attention over its legal keys in the retained tiles."""
+    G, Nk, d, B = 3, 48, 4, 8
+    rng = np.random.default_rng(seed)
+    Qg = rng.standard_normal((G, Nq, d)) * 5 / 2
+    K = rng.standard_normal((Nk, d))
+    V = rng.standard_normal((Nk, d))
+    O, z, keep, _ = orc.forward_group(Qg, K, V, B, B, tau)
+    off = Nk - Nq
+    nQB, nKB = -(-Nq // B), -(-Nk // B)
+    skipped = 0
+    for i in range(nQB):
+        rows = range(i * B, min((i + 1) * B, Nq))
+        j_diag = (rows[-1] + off) // B
+        kept_tiles = []
+        for j in range(j_diag, -1, -1):
+            want = False
+            for g in range(G):
+                for r in rows:
+                    p = r + off
+                    legal = [k for k in range(j * B, min((j + 1) * B, Nk)) if k <= p]
+                    if not legal:
+                        continue
+                    mine = [k for t in kept_tiles for k in range(t * B, min((t + 1) * B, Nk)) if k <= p]
+                    if not mine:
+                        want = True
+                        continue
+                    mass = sum(math.exp(Qg[g, r] @ K[k]) for k in mine)
+                    best = max(math.exp(Qg[g, r] @ K[k]) for k in legal)
+                    if best / mass >= tau / (p + 1):
+                        want = True
+            assert keep[i, j] == want, (i, j)
+            if want:
+                kept_tiles.append(j)
+            else:
+                skipped += 1
+        for g in range(G):
+            for r in rows:
+                p = r + off
+                ks = [k for t in kept_tiles for k in range(t * B, min((t + 1) * B, Nk)) if k <= p]
+                w = np.array([math.exp(Qg[g, r] @ K[k]) for k in ks])
+                assert np.allclose(O[g, r], (w / w.sum()) @ V[ks], atol=1e-11)
+                assert abs(z[g, r] - math.log(w.sum())) < 1e-11
+    if tau >= 100.0:
+        assert skipped > 0                           # the case does skip
+
+
 def test_replay_forces_decisions_but_keeps_margins():
     Q, K, V = _rand_case(41, 32, 4, sharp=5.0)
     O, z, keep, margin = orc.forward_head(Q, K, V, 8, 8, 0.5)
