@@ -127,6 +127,16 @@ typedef struct {
    * only (bf16, 128 x 128 tiles); at most MALA_MAX_SEQS sequences. */
   const int32_t* cu_seqlens_q;
   const int32_t* cu_seqlens_k;
+  /* 0 (the default): every query head decides for itself. 1: group-joint
+   * voting, one decision per (query block, key tile) for the G = H_q / H_kv
+   * query heads of a KV head: their rows of the block are treated like the
+   * rows of one query block, so a tile is skipped only when every row of
+   * every head passes the skip test, and a retained tile is accumulated by
+   * every head. keep_mask bits are then equal across a group, and mala_bwd
+   * replays them as usual. Tensor-core path only (bf16, 128 x 128 tiles),
+   * the default head map (q_to_kv NULL or h -> h / G) and G <= 8, else
+   * MALA_ERR_UNSUPPORTED; other values MALA_ERR_INVALID_ARG. */
+  int32_t group_vote;
 } mala_fwd_args;
 
 #define MALA_MAX_SEQS 128

@@ -211,6 +211,49 @@ def check_decode_group(q, k, v, o, lse, keep_words, tau, P, B_k=128, groups=None
     return rep
 
 
+def check_fwd_group(q, k, v, o, lse, keep_words, tau, groups=None, B_q=128, B_k=128):
+    """mala_fwd(group_vote=True) vs the oracle's group-joint prefill for
+    (batch, KV head) pairs ``groups`` (None = all), default head map, all
+    query blocks. The heads of a group must carry identical keep bits; a
+    decision that differs from the oracle's must lie inside the margin band
+    (the oracle then replays the GPU's decisions); O and LSE of every row of
+    every head must match. Returns (blocks, tiles visited, tiles kept)."""
+    B, N, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    nQB, nKB = orc.num_blocks(N, B_q), orc.num_blocks(Nk, B_k)
+    keep = mala.unpack_mask(keep_words, nKB)             # [B, Hq, nQB, nKB]
+    if groups is None:
+        groups = [(b, hk) for b in range(B) for hk in range(Hkv)]
+    o_c, lse_c = f64(o), lse.detach().cpu().numpy()
+    q64, k64, v64 = f64(q), f64(k), f64(v)
+    nblk = ntiles = nkept = 0
+    for (b, hk) in groups:
+        h0 = hk * G
+        gk = np.asarray(keep[b, h0], dtype=bool)
+        for h in range(h0 + 1, h0 + G):
+            assert (np.asarray(keep[b, h], dtype=bool) == gk).all(), \
+                f"group b={b} hk={hk}: heads {h0} and {h} carry different keep bits"
+        Qg = np.stack([q64[b, :, h0 + g] for g in range(G)])
+        K, V = k64[b, :, hk], v64[b, :, hk]
+        O, z, okeep, margin = orc.forward_group(Qg, K, V, B_q, B_k, tau)
+        visited = ~np.isnan(margin)
+        if (okeep[visited] != gk[visited]).any():
+            O, z, okeep, margin = orc.forward_group(Qg, K, V, B_q, B_k, tau, replay_mask=gk)
+        for (i, j) in zip(*np.nonzero(visited)):
+            if gk[i, j] != (margin[i, j] <= 0.0):
+                assert abs(margin[i, j]) <= MARGIN_BAND, \
+                    f"group b={b} hk={hk} block {i} tile {j}: decided {gk[i, j]} with margin {margin[i, j]:.3e}"
+        assert not gk[~visited].any(), f"group b={b} hk={hk}: bits set on tiles never visited"
+        for g in range(G):
+            assert_close(o_c[b, :, h0 + g], O[g], f"group fwd b={b} h={h0 + g} O")
+            assert_close(lse_c[b, h0 + g], z[g], f"group fwd b={b} h={h0 + g} LSE")
+        nblk += nQB
+        ntiles += int(visited.sum())
+        nkept += int(gk[visited].sum())
+    return nblk, ntiles, nkept
+
+
 def oracle_forward_replaying(q64, k64, v64, b, h, G, blocks, gpu_keep_bh, B_q, B_k, tau, rep=None):
     """Oracle O and z for query blocks ``blocks`` of head (b, h), with the
     GPU's forward decisions forced; every forced decision that differs from
@@ -248,11 +291,13 @@ def as_operator_outputs(O, z):
 
 
 def check_bwd_blocks(q, k, v, do, fwd_keep_words, bwd_keep_words, dq, dk, dv, tau,
-                     kv_samples=None, q_samples=None, B_q=128, B_k=128):
+                     kv_samples=None, q_samples=None, B_q=128, B_k=128, group_vote=False):
     """Backward parity. kv_samples: (b, hk, j) key blocks whose dK/dV rows are
     checked (None = all); q_samples: (b, h, i) query blocks whose dQ rows are
     checked (None = all). Gradients by relative Frobenius error per block;
-    backward decisions by the margin band."""
+    backward decisions by the margin band. group_vote: the forward mask came
+    from group-joint voting, so the oracle's forward outputs are those of its
+    group-joint prefill replaying that mask (default head map)."""
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
     G = Hq // Hkv
@@ -273,7 +318,24 @@ def check_bwd_blocks(q, k, v, do, fwd_keep_words, bwd_keep_words, dq, dk, dv, ta
     err2 = {"dQ": 0.0, "dK": 0.0, "dV": 0.0}
     ref2 = {"dQ": 0.0, "dK": 0.0, "dV": 0.0}
 
+    def fwd_rows_group(b, h):
+        if (b, h) not in cache:
+            hk = h // G
+            h0 = hk * G
+            gm = np.asarray(fkeep[b, h0], dtype=bool)
+            Qg = np.stack([q64[b, :, h0 + g] for g in range(G)])
+            O, z, _, margin = orc.forward_group(Qg, k64[b, :, hk], v64[b, :, hk], B_q, B_k, tau, replay_mask=gm)
+            for (i, j) in zip(*np.nonzero(~np.isnan(margin))):
+                if gm[i, j] != (margin[i, j] <= 0.0):
+                    assert abs(margin[i, j]) <= MARGIN_BAND, \
+                        f"group fwd b={b} hk={hk} tile ({i},{j}): margin {margin[i, j]:.3e}"
+            for g in range(G):
+                cache[(b, h0 + g)] = (O[g], z[g])
+        return as_operator_outputs(*cache[(b, h)])
+
     def fwd_rows(b, h, blocks):
+        if group_vote:
+            return fwd_rows_group(b, h)
         key = (b, h)
         O, z = cache.get(key, (None, None))
         need = [i for i in blocks if O is None or np.isnan(z[i * B_q])]

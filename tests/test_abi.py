@@ -228,3 +228,22 @@ def test_decode_rejects_bad_arguments_without_launching(lib, kw):
     assert lib.mala_decode_workspace_size(ctypes.byref(a)) == 0
     assert lib.mala_decode(ctypes.byref(a), None, 0, None) == mala.MALA_ERR_INVALID_ARG
     assert lib.mala_last_error_message().decode()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(group_vote=2), mala.MALA_ERR_INVALID_ARG),
+    (dict(group_vote=1, dtype=mala.MALA_FP32), mala.MALA_ERR_UNSUPPORTED),
+    (dict(group_vote=1, block_q=64, block_k=64), mala.MALA_ERR_UNSUPPORTED),
+    (dict(group_vote=1, heads_q=32, heads_kv=2,
+          q_stride=mala._i64x3(256 * 32 * 128, 32 * 128, 128)), mala.MALA_ERR_UNSUPPORTED),   # G = 16
+])
+def test_fwd_group_vote_rejections(lib, kw, code):
+    a = _fwd_args(**kw)
+    assert lib.mala_fwd(ctypes.byref(a), None, 0, None) == code, lib.mala_last_error_message()
+
+
+def test_fwd_group_vote_needs_the_default_head_map(lib):
+    arr = (ctypes.c_int32 * 4)(1, 0, 0, 1)          # valid, but not h -> h / 2
+    a = _fwd_args(group_vote=1, q_to_kv=ctypes.cast(arr, ctypes.c_void_p))
+    assert lib.mala_fwd(ctypes.byref(a), None, 0, None) == mala.MALA_ERR_UNSUPPORTED
+    assert "head map" in lib.mala_last_error_message().decode()

@@ -22,6 +22,13 @@
 //              with P read straight from TMEM.
 // TMEM: S buffers at cols [0,128), [128,256), [256,384); O = [384, 384 + D).
 //
+// Group-joint voting (optional): the G CTAs that hold the same query block
+// of the G query heads of one KV head run as one thread-block cluster. After
+// its own vote, each CTA writes it into every peer's shared memory and
+// arrives on the peer's vote barrier; each then takes the OR of the G votes,
+// so the group keeps or skips a tile together (the heads' rows act as the
+// rows of one block). Votes alternate between two slots by tile parity.
+//
 // Numerics: scores are accumulated in fp32 from bf16 operands. The online
 // state is kept in base 2: m2 is a reference maximum (in log2 units) and l
 // the sum of 2^(s*log2e - m2) over retained keys, so log Z = (m2 + log2 l)
@@ -82,7 +89,9 @@ struct Layout {
   static constexpr uint32_t kXSum = kX + 2 * 2 * 128 * 4;           // [2 parity][2 groups][128] float
   static constexpr uint32_t kBars = kXSum + 2 * 2 * 128 * 4;
   static constexpr uint32_t kMisc = kBars + kNumBars * 8;
-  static constexpr uint32_t kEnd = kMisc + 64;
+  static constexpr uint32_t kCVote = kMisc + 64;                    // [2 parity][8 ranks] uint32 group votes
+  static constexpr uint32_t kCBars = kCVote + 2 * 8 * 4;            // 2 vote barriers (G arrivals each)
+  static constexpr uint32_t kEnd = kCBars + 2 * 8;
   static constexpr uint32_t kAlloc = kEnd + 1024;  // slack for 1024-byte alignment
 };
 
@@ -115,6 +124,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
   float* xsum = reinterpret_cast<float*>(smem + L::kXSum);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L::kMisc);
+  volatile uint32_t* cvote = reinterpret_cast<volatile uint32_t*>(smem + L::kCVote);
+  uint64_t* cbars = reinterpret_cast<uint64_t*>(smem + L::kCBars);
   // misc[0] TMEM base, misc[1] abort flag, misc[2..4] progress markers of the
   // producer / MMA / softmax roles (kept for timeout diagnosis), misc[5..6]
   // decisions of tiles t & 1
@@ -165,6 +176,10 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       if (x == kDecEmpty || x == kDecEmpty + 1) cnt = 2;
       mbar_init(&bars[x], cnt);
     }
+    if (p.group_vote) {
+      mbar_init(&cbars[0], p.group);
+      mbar_init(&cbars[1], p.group);
+    }
     for (int x = 1; x < 16; ++x) misc[x] = 0;
     fence_mbar_init();
   }
@@ -175,6 +190,10 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // every CTA of the cluster has initialised its vote barriers before any
+  // peer arrives on them
+  if (p.group_vote) cluster_sync_all();
+  const uint32_t crank = p.group_vote ? cluster_ctarank() : 0u;
   const uint32_t tmem = misc[0];
   const uint32_t tmem_o = tmem + kNS * 128;
 
@@ -375,7 +394,26 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       // retain iff the row's largest contribution ratio reaches tau / L_q;
       // an empty retained set (l = 0) always retains
       const bool vote = has_key && (l == 0.0f || rmax2 - (m2 + lg2_approx(l)) >= thr2);
-      const bool keep = bar_or(1, 256, vote);
+      bool keep = bar_or(1, 256, vote);
+      if (p.group_vote) {
+        // group-joint voting: send this block's vote to every CTA of the
+        // cluster, then OR the G votes of tile t. A slot of parity par is
+        // rewritten (tile t + 2) only after every peer has passed the tile
+        // t + 1 exchange, hence after this CTA read it.
+        if (tid == 0) {
+          const uint32_t slot = smem_u32(const_cast<uint32_t*>(&cvote[par * 8 + crank]));
+          const uint32_t cbar = smem_u32(&cbars[par]);
+          for (int rr = 0; rr < p.group; ++rr) {
+            st_cluster_u32(mapa_shared(slot, rr), keep ? 1u : 0u);
+            mbar_arrive_cluster(mapa_shared(cbar, rr));
+          }
+        }
+        if (mbar_wait<true>(&cbars[par], (t >> 1) & 1, abort_flag, p.err, wait_tag(0, 0x40 + par, t))) {
+          bool any = false;
+          for (int rr = 0; rr < p.group; ++rr) any = any || cvote[par * 8 + rr] != 0u;
+          keep = any;
+        }
+      }
 
       if (tid == 0) {
         if (mbar_wait(&bars[kDecEmpty + par], ((t >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty + par, t))) {
@@ -510,6 +548,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // no CTA leaves while a peer may still write to its shared memory
+  if (p.group_vote) cluster_sync_all();
 }
 
 }  // namespace
@@ -518,20 +558,42 @@ size_t fwd_tc_smem_bytes(int head_dim) {
   return head_dim == 64 ? Layout<64>::kAlloc : Layout<128>::kAlloc;
 }
 
+// Group-joint voting: clusters of G consecutive CTAs, which the work-item
+// order makes the G query heads of one KV head on the same query block.
+template <int D>
+cudaError_t launch_fwd_tc_clustered(const FwdTcParams& p, unsigned grid, int smem, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(p.group);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mala_fwd_tc_kernel<D>, p);
+}
+
 cudaError_t launch_fwd_tc(const FwdTcParams& p, int head_dim, cudaStream_t stream) {
   const unsigned grid = static_cast<unsigned>(p.B) * p.Hq * p.nQB;
   if (grid == 0) return cudaSuccess;
+  if (p.group_vote && (p.group < 1 || p.group > 8 || p.Hq % p.group != 0)) return cudaErrorInvalidValue;
   if (head_dim == 128) {
     const int smem = Layout<128>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(mala_fwd_tc_kernel<128>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    if (p.group_vote) return launch_fwd_tc_clustered<128>(p, grid, smem, stream);
     mala_fwd_tc_kernel<128><<<grid, kThreads, smem, stream>>>(p);
   } else {
     const int smem = Layout<64>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(mala_fwd_tc_kernel<64>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    if (p.group_vote) return launch_fwd_tc_clustered<64>(p, grid, smem, stream);
     mala_fwd_tc_kernel<64><<<grid, kThreads, smem, stream>>>(p);
   }
   return cudaGetLastError();

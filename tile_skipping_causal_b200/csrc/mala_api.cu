@@ -267,10 +267,23 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
   const bool tc = a->dtype == MALA_BF16 && a->block_q == 128 && a->block_k == 128;
+  if (a->group_vote != 0 && a->group_vote != 1)
+    return fail(MALA_ERR_INVALID_ARG, "group_vote %d is neither 0 nor 1", a->group_vote);
+  if (a->group_vote && !tc)
+    return fail(MALA_ERR_UNSUPPORTED, "group-joint voting needs the tensor-core path (bf16, 128 x 128 tiles)");
   if (tc) {
     mala::FwdTcParams p;
     memset(&p, 0, sizeof(p));
     if ((rc = head_map(a->q_to_kv, a->heads_q, a->heads_kv, p.kv_of_q))) return rc;
+    if (a->group_vote) {
+      const int G = static_cast<int>(a->heads_q / a->heads_kv);
+      if (G > 8) return fail(MALA_ERR_UNSUPPORTED, "group-joint voting supports groups of at most 8 query heads");
+      for (int64_t h = 0; h < a->heads_q; ++h)
+        if (p.kv_of_q[h] != h / G)
+          return fail(MALA_ERR_UNSUPPORTED, "group-joint voting needs the default head map (h -> h / G)");
+      p.group_vote = 1;
+      p.group = G;
+    }
     // packed sequences: one batch entry of total_q / total_k rows
     const int64_t mb = packed ? 1 : a->batch;
     if ((rc = make_map_bf16(&p.tm_q, a->q, mb, N, a->heads_q, d, a->q_stride, 128))) return rc;

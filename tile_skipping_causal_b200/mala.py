@@ -36,6 +36,7 @@ class FwdArgs(ctypes.Structure):
         ("q_to_kv", ctypes.c_void_p), ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32),
         ("tau", ctypes.c_float), ("dtype", ctypes.c_int32), ("mode", ctypes.c_int32),
         ("stats", ctypes.c_void_p), ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+        ("group_vote", ctypes.c_int32),
     ]
 
 
@@ -235,7 +236,7 @@ def _packed(cu_seqlens_q, cu_seqlens_k, block_q, block_k):
 def mala_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float,
              block_q: int = 128, block_k: int = 128, *, o=None, lse=None, keep_mask=None,
              with_mask: bool = True, stats=None, q_to_kv=None, stream=None,
-             cu_seqlens_q=None, cu_seqlens_k=None):
+             cu_seqlens_q=None, cu_seqlens_k=None, group_vote: bool = False):
     """MALA forward/prefill. q [B, N_q, Hq, d], k/v [B, N_k, Hkv, d] (bf16 or
     fp32, scale folded into q; N_q <= N_k, bottom-right aligned). Returns
     (o, lse [B, Hq, N_q] fp32, keep_mask words [B, Hq, nQB, ceil(nKB/32)]
@@ -244,7 +245,12 @@ def mala_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float,
     Packed sequences: cu_seqlens_q / cu_seqlens_k (host int32 offsets, one
     more than the number of sequences) with q [1, total_q, Hq, d] and k, v
     [1, total_k, Hkv, d]; lse is then [Hq, total_q] and keep_mask
-    [Hq, packed query blocks, ceil(largest key-block count / 32)]."""
+    [Hq, packed query blocks, ceil(largest key-block count / 32)].
+
+    group_vote: one decision per (query block, key tile) for the query heads
+    of a KV head (a tile is skipped only when every row of every head passes
+    the test; bf16, 128 x 128 tiles, default head map, at most 8 heads per
+    group)."""
     lib = load_library()
     _require_cuda(q, k, v)
     B, N, Hq, d = q.shape
@@ -264,6 +270,7 @@ def mala_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float,
         keep_mask = torch.empty(shape, dtype=torch.int32, device=q.device)
     keep_alive, hm = _head_map(q_to_kv)
     a = fwd_args(q, k, v, o, lse, keep_mask, tau, block_q, block_k, stats, hm)
+    a.group_vote = 1 if group_vote else 0
     if packed:
         a.batch = packed[2]
         a.cu_seqlens_q = packed[0].ctypes.data
