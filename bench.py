@@ -344,6 +344,7 @@ def run_mala(args):
 
     peaks = _peaks()
     chunk = bench_chunk(args, q, k, v, stream, peaks)
+    grp = None if args.no_extras else bench_group_fwd(args, q, k, v, stream, peaks)
     dec = None if args.no_decode else bench_decode(args, dev, stream, peaks)
     dec8 = None if args.no_decode else bench_decode(args, dev, stream, peaks, e4m3=True)
     kern_f = statistics.mean(fwd_times)
@@ -394,6 +395,8 @@ def run_mala(args):
         "clocks": clk.summary(),
     }
     res["chunked_prefill"] = chunk
+    if grp is not None:
+        res["fwd_group_vote"] = grp
     if dec is not None:
         res["decode"] = dec
         res["decode_e4m3"] = dec8
@@ -438,6 +441,46 @@ def bench_chunk(args, q, k, v, stream, peaks, chunk: int = 4096):
     return {"seqlen_q": chunk, "seqlen_k": Nk, "tau": TAU, "ms": t * 1e3,
             "tokens_per_s": q.shape[0] * chunk / t, "tiles_tested": tested, "tiles_kept": kept,
             "tflops_executed": flops / t / 1e12, "frac_of_peak": flops / t / 1e12 / peak}
+
+
+def bench_group_fwd(args, q, k, v, stream, peaks, taus=(TAU, 64.0)):
+    """The forward of the workload with group-joint voting (the query heads
+    of a KV head decide together per tile), and per-head voting beside it, at
+    each tau: device time per call, tiles tested / kept per head, executed
+    FLOPs as for the step's forward."""
+    import torch
+    from tile_skipping_causal_b200 import mala
+
+    B, N, Hq, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    out = {}
+    for tau in taus:
+        row = {}
+        for mode in ("group", "per_head"):
+            gv = mode == "group"
+            stats = torch.zeros(4, dtype=torch.int64, device=q.device)
+            keep = mala.mala_fwd(q, k, v, tau, TILE, TILE, o=o, lse=lse, stats=stats, group_vote=gv)[2]
+            mala.check_device_error()
+            tested, kept = (int(x) for x in stats.cpu().tolist()[:2])
+            for _ in range(max(3, args.warmup)):
+                mala.mala_fwd(q, k, v, tau, TILE, TILE, o=o, lse=lse, keep_mask=keep, group_vote=gv)
+            torch.cuda.synchronize()
+            n = max(5, args.steps // 2)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                mala.mala_fwd(q, k, v, tau, TILE, TILE, o=o, lse=lse, keep_mask=keep, group_vote=gv)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            mala.check_device_error()
+            t = e0.elapsed_time(e1) / 1e3 / n
+            flops = tile_flops(d) * (tested + kept)
+            row[mode] = {"ms": t * 1e3, "tiles_tested": tested, "tiles_kept": kept,
+                         "kept_fraction": kept / tested, "tflops_executed": flops / t / 1e12,
+                         "frac_of_peak": flops / t / 1e12 / peaks["bf16_tflops_sustained"]}
+        out[str(tau)] = row
+    return out
 
 
 def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072, e4m3: bool = False):
@@ -633,12 +676,23 @@ def main():
                     help="run only the decode measurement (profiling captures)")
     ap.add_argument("--decode-e4m3", action="store_true",
                     help="with --decode-only: an e4m3 cache instead of bf16")
+    ap.add_argument("--group-only", action="store_true",
+                    help="run only the group-joint voting forward measurement")
     ap.add_argument("--no-extras", action="store_true",
                     help="time the step only (no tau=0, e2e, baseline); for profiling captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         run_reference(args)
+    elif args.group_only:
+        import torch
+        from tile_skipping_causal_b200 import mala, synth
+        mala.load_library()
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        t = synth.make_prefill(synth.WORKLOADS[WORKLOAD], SEED, seqlen=args.seqlen)
+        q, k, v = (t[n].to(dev) for n in ("q", "k", "v"))
+        print(json.dumps(bench_group_fwd(args, q, k, v, torch.cuda.current_stream(), _peaks())), flush=True)
     elif args.decode_only:
         import torch
         from tile_skipping_causal_b200 import mala
