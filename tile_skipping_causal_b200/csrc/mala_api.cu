@@ -565,28 +565,12 @@ size_t decode_ws_bytes(const mala_decode_args* a, int P) {
   return static_cast<size_t>(a->batch) * a->heads_q * P * (128 + 1) * sizeof(float) + 256;
 }
 
-}  // namespace
-
-size_t mala_decode_workspace_size(const mala_decode_args* a) {
-  if (!a) return 0;
-  int nKB = 0;
-  if (decode_check(a, &nKB) != MALA_OK) return 0;
-  const int P = a->num_splits > 0 ? a->num_splits : choose_splits(a->batch * a->heads_kv, nKB);
-  return decode_ws_bytes(a, P);
-}
-
-int mala_decode(mala_decode_args* a, void* workspace, size_t ws_bytes, void* stream_) {
-  g_msg[0] = 0;
-  if (!a) return fail(MALA_ERR_INVALID_ARG, "args is NULL");
-  int nKB = 0;
-  int rc = decode_check(a, &nKB);
-  if (rc) return rc;
-  const int P = a->num_splits > 0 ? a->num_splits : choose_splits(a->batch * a->heads_kv, nKB);
-  const size_t need = decode_ws_bytes(a, P);
-  if (need > 0 && (!workspace || ws_bytes < need))
-    return fail(MALA_ERR_WORKSPACE, "decode workspace of %zu bytes needed", need);
-  if (need > 0 && !aligned16(workspace)) return fail(MALA_ERR_INVALID_ARG, "workspace misaligned");
-
+// Fills the decode kernel parameters of a checked call and launches it on
+// the caller's stream. partials: [B, H_q, P, 128] + [B, H_q, P] fp32 when
+// P > 1 (unused otherwise); it needs no clearing, since every split writes
+// all of its rows before the merge kernel reads them.
+int decode_launch(mala_decode_args* a, int nKB, int P, float* partials, void* stream_) {
+  int rc;
   mala::DecodeParams p;
   memset(&p, 0, sizeof(p));
   uint8_t kv_of_q[mala::kMaxHeads];
@@ -607,8 +591,8 @@ int mala_decode(mala_decode_args* a, void* workspace, size_t ws_bytes, void* str
   p.keep_mask = a->keep_mask;
   p.stats = a->stats;
   if (P > 1) {
-    p.part_o = static_cast<float*>(workspace);
-    p.part_lse = p.part_o + static_cast<size_t>(a->batch) * a->heads_q * P * 128;
+    p.part_o = partials;
+    p.part_lse = partials + static_cast<size_t>(a->batch) * a->heads_q * P * 128;
   }
   p.q_sb = a->q_stride[0];
   p.q_sh = a->q_stride[2];
@@ -632,6 +616,31 @@ int mala_decode(mala_decode_args* a, void* workspace, size_t ws_bytes, void* str
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   a->num_splits = P;
   return MALA_OK;
+}
+
+}  // namespace
+
+size_t mala_decode_workspace_size(const mala_decode_args* a) {
+  if (!a) return 0;
+  int nKB = 0;
+  if (decode_check(a, &nKB) != MALA_OK) return 0;
+  const int P = a->num_splits > 0 ? a->num_splits : choose_splits(a->batch * a->heads_kv, nKB);
+  return decode_ws_bytes(a, P);
+}
+
+int mala_decode(mala_decode_args* a, void* workspace, size_t ws_bytes, void* stream_) {
+  g_msg[0] = 0;
+  if (!a) return fail(MALA_ERR_INVALID_ARG, "args is NULL");
+  int nKB = 0;
+  int rc = decode_check(a, &nKB);
+  if (rc) return rc;
+  const int P = a->num_splits > 0 ? a->num_splits : choose_splits(a->batch * a->heads_kv, nKB);
+  const size_t need = decode_ws_bytes(a, P);
+  if (need > 0 && (!workspace || ws_bytes < need))
+    return fail(MALA_ERR_WORKSPACE, "decode workspace of %zu bytes needed", need);
+  if (need > 0 && !aligned16(workspace)) return fail(MALA_ERR_INVALID_ARG, "workspace misaligned");
+
+  return decode_launch(a, nKB, P, static_cast<float*>(workspace), stream_);
 }
 
 }  // extern "C"
@@ -688,52 +697,5 @@ extern "C" int mala_decode_noalloc(mala_decode_args* a, void* stream_) {
     scratch = decode_noalloc_scratch();
     if (!scratch) return fail(MALA_ERR_CUDA, "cannot resolve the built-in decode scratch buffer");
   }
-
-  mala::DecodeParams p;
-  memset(&p, 0, sizeof(p));
-  uint8_t kv_of_q[mala::kMaxHeads];
-  if ((rc = head_map(a->q_to_kv, a->heads_q, a->heads_kv, kv_of_q))) return rc;
-  for (int64_t h = 0; h < a->heads_q; ++h) {
-    const int hk = kv_of_q[h];
-    if (p.group_size[hk] >= mala::kMaxGroup)
-      return fail(MALA_ERR_UNSUPPORTED, "more than %d query heads share KV head %d", mala::kMaxGroup, hk);
-    p.group_heads[hk][p.group_size[hk]++] = static_cast<uint8_t>(h);
-  }
-  if ((rc = decode_cache_maps(a, &p))) return rc;
-  p.group_vote = a->group_vote;
-  p.err = device_error_ptr();
-  if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
-  p.q = a->q;
-  p.o = a->o;
-  p.lse = a->lse;
-  p.keep_mask = a->keep_mask;
-  p.stats = a->stats;
-  if (P > 1) {
-    // the partials need no clearing: every split writes all of its rows
-    // before the merge kernel reads them
-    p.part_o = scratch;
-    p.part_lse = scratch + static_cast<size_t>(a->batch) * a->heads_q * P * 128;
-  }
-  p.q_sb = a->q_stride[0];
-  p.q_sh = a->q_stride[2];
-  p.o_sb = a->o_stride[0];
-  p.o_sh = a->o_stride[2];
-  p.B = static_cast<int>(a->batch);
-  p.Hq = static_cast<int>(a->heads_q);
-  p.Hkv = static_cast<int>(a->heads_kv);
-  p.Nk = static_cast<int>(a->seqlen_k);
-  p.nKB = nKB;
-  p.mask_words = (nKB + 31) / 32;
-  p.num_splits = P;
-  p.log2_tau = a->tau == 0.0f ? -INFINITY : log2f(a->tau);
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  if (a->keep_mask) {
-    cudaError_t e = cudaMemsetAsync(a->keep_mask, 0,
-                                    static_cast<size_t>(a->batch) * a->heads_q * p.mask_words * 4, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "keep mask clear");
-  }
-  cudaError_t e = mala::launch_decode(p, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  a->num_splits = P;
-  return MALA_OK;
+  return decode_launch(a, nKB, P, scratch, stream_);
 }
