@@ -247,3 +247,21 @@ def test_fwd_group_vote_needs_the_default_head_map(lib):
     a = _fwd_args(group_vote=1, q_to_kv=ctypes.cast(arr, ctypes.c_void_p))
     assert lib.mala_fwd(ctypes.byref(a), None, 0, None) == mala.MALA_ERR_UNSUPPORTED
     assert "head map" in lib.mala_last_error_message().decode()
+
+
+def test_binding_refuses_host_tensors(lib):
+    """No CPU fallback: every entry point raises on host tensors."""
+    import torch
+    q = torch.zeros(1, 128, 4, 128, dtype=torch.bfloat16)
+    k = torch.zeros(1, 128, 2, 128, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 4, 128)
+    keep = torch.zeros(1, 4, 1, 1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        mala.mala_fwd(q, k, k, 0.1)
+    with pytest.raises(ValueError, match="CUDA"):
+        mala.mala_bwd(q, k, k, q, q, lse, 0.1, keep)
+    q1 = q[:, :1]
+    with pytest.raises(ValueError, match="CUDA"):
+        mala.mala_decode(q1, k, k, 0.1)
+    with pytest.raises(ValueError, match="CUDA"):
+        mala.mala_decode_noalloc(q1, k, k, 0.1, group_vote=True)

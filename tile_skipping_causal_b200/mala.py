@@ -343,17 +343,10 @@ def _decode_cache(a, k, v, k_scale, v_scale):
     a.k_scale, a.v_scale = float(k_scale), float(v_scale)
 
 
-def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *, o=None,
-                lse=None, keep_mask=None, with_mask: bool = True, stats=None, q_to_kv=None,
-                stream=None, workspace=None, k_scale: float = 1.0, v_scale: float = 1.0,
-                group_vote: bool = False):
-    """Single-token decoding. q [B, 1, Hq, d] bf16; k/v cache [B, Nk, Hkv, d]
-    in bf16, or torch.float8_e4m3fn codes whose values are code * k_scale and
-    code * v_scale. group_vote: one decision per key tile for all query heads
-    of a KV head (a tile is skipped only when every head passes the test).
-    Returns (o, lse [B, Hq], keep_mask words [B, Hq, ceil(T/32)] or None,
-    num_splits used)."""
-    lib = load_library()
+def _decode_call(q, k, v, tau, block_k, num_splits, o, lse, keep_mask, with_mask, stats, q_to_kv,
+                 k_scale, v_scale, group_vote):
+    """Output tensors and the filled argument struct of a decode call (plus
+    the objects that must outlive the call)."""
     _require_cuda(q, k, v)
     B, _, Hq, d = q.shape
     _, Nk, Hkv, _ = k.shape
@@ -376,6 +369,22 @@ def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *,
     a.stats = _ptr(stats)
     _decode_cache(a, k, v, k_scale, v_scale)
     a.group_vote = 1 if group_vote else 0
+    return o, lse, keep_mask, a, keep_alive
+
+
+def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *, o=None,
+                lse=None, keep_mask=None, with_mask: bool = True, stats=None, q_to_kv=None,
+                stream=None, workspace=None, k_scale: float = 1.0, v_scale: float = 1.0,
+                group_vote: bool = False):
+    """Single-token decoding. q [B, 1, Hq, d] bf16; k/v cache [B, Nk, Hkv, d]
+    in bf16, or torch.float8_e4m3fn codes whose values are code * k_scale and
+    code * v_scale. group_vote: one decision per key tile for all query heads
+    of a KV head (a tile is skipped only when every head passes the test).
+    Returns (o, lse [B, Hq], keep_mask words [B, Hq, ceil(T/32)] or None,
+    num_splits used)."""
+    lib = load_library()
+    o, lse, keep_mask, a, keep_alive = _decode_call(q, k, v, tau, block_k, num_splits, o, lse, keep_mask,
+                                                    with_mask, stats, q_to_kv, k_scale, v_scale, group_vote)
     ws_n = lib.mala_decode_workspace_size(ctypes.byref(a))
     own_ws = workspace is None or workspace.numel() < ws_n
     if own_ws:
@@ -396,28 +405,8 @@ def mala_decode_noalloc(q, k, v, tau: float, block_k: int = 128, num_splits: int
     calls that overlap on the GPU race on that buffer). Returns the same
     tuple as :func:`mala_decode`."""
     lib = load_library()
-    _require_cuda(q, k, v)
-    B, _, Hq, d = q.shape
-    _, Nk, Hkv, _ = k.shape
-    nKB = -(-Nk // block_k)
-    o = torch.empty_like(q) if o is None else o
-    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
-    if keep_mask is None and with_mask:
-        keep_mask = torch.empty((B, Hq, mask_words(nKB)), dtype=torch.int32, device=q.device)
-    keep_alive, hm = _head_map(q_to_kv)
-    a = DecodeArgs()
-    a.q, a.k, a.v, a.o = _ptr(q), _ptr(k), _ptr(v), _ptr(o)
-    a.lse, a.keep_mask = _ptr(lse), _ptr(keep_mask)
-    a.batch, a.heads_q, a.heads_kv, a.seqlen_k, a.head_dim = B, Hq, Hkv, Nk, d
-    a.q_stride, a.k_stride, a.v_stride, a.o_stride = _strides(q), _strides(k), _strides(v), _strides(o)
-    a.q_to_kv = hm
-    a.block_k = block_k
-    a.tau = float(tau)
-    a.dtype = _dtype_code(q)
-    a.num_splits = int(num_splits)
-    a.stats = _ptr(stats)
-    _decode_cache(a, k, v, k_scale, v_scale)
-    a.group_vote = 1 if group_vote else 0
+    o, lse, keep_mask, a, keep_alive = _decode_call(q, k, v, tau, block_k, num_splits, o, lse, keep_mask,
+                                                    with_mask, stats, q_to_kv, k_scale, v_scale, group_vote)
     _check(lib.mala_decode_noalloc(ctypes.byref(a), _stream(stream)))
     del keep_alive
     return o, lse, keep_mask, int(a.num_splits)
