@@ -209,7 +209,8 @@ MALA_API int mala_bwd(const mala_bwd_args* args, void* workspace, size_t workspa
  * [floor(p*T/P), floor((p+1)*T/P)); each split visits its tiles in
  * descending order with its own running maximum and normalisation sum, and
  * tests every tile against tau / N_k. A tile's V is read iff some query
- * head of the group retains it; PV runs only for the retaining heads. The
+ * head of the group retains it; PV runs only for the retaining heads (for
+ * every head of the group with group_vote = 1). The
  * partial outputs are merged by their log-normalisers:
  * z = log sum_p exp(z_p), O = sum_p exp(z_p - z) O_p.
  *
@@ -217,7 +218,8 @@ MALA_API int mala_bwd(const mala_bwd_args* args, void* workspace, size_t workspa
  * fp32; keep_mask optional [B, H_q, ceil(T/32)] uint32.
  * num_splits: in 0 = let the library choose, else the requested P
  * (1 <= P <= T); out: the P used (host-side value, known before launch).
- * Supported: MALA_BF16, d = 128, B_k = 128, H_q / H_kv <= 16.
+ * Supported: q in MALA_BF16, the K / V cache in MALA_BF16 or
+ * MALA_FP8_E4M3 (kv_dtype), d = 128, B_k = 128, H_q / H_kv <= 16.
  */
 typedef struct {
   const void* q;
