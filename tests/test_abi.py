@@ -265,3 +265,35 @@ def test_binding_refuses_host_tensors(lib):
         mala.mala_decode(q1, k, k, 0.1)
     with pytest.raises(ValueError, match="CUDA"):
         mala.mala_decode_noalloc(q1, k, k, 0.1, group_vote=True)
+
+
+def test_c_program_links_and_runs(lib):
+    """A plain C consumer: compiles against include/mala.h, links libmala.so
+    and calls the host-only entry points (no GPU needed). An argument error
+    comes back as a status code with a message, before anything launches."""
+    prog = r'''
+#include <stdio.h>
+#include <string.h>
+#include "mala.h"
+int main(void) {
+  mala_decode_args a;
+  memset(&a, 0, sizeof(a));
+  int rc = mala_decode(&a, NULL, 0, NULL);          /* NULL tensors: rejected on the host */
+  printf("%s %s %d %s\n", mala_version(), mala_status_string(MALA_ERR_TIMEOUT), rc,
+         mala_last_error_message()[0] ? "msg" : "nomsg");
+  printf("%zu\n", mala_decode_workspace_size(&a));
+  return rc == MALA_ERR_INVALID_ARG ? 0 : 1;
+}
+'''
+    libdir = os.path.dirname(mala.LIB_PATH)
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "consumer.c")
+        exe = os.path.join(d, "consumer")
+        open(c, "w").write(prog)
+        subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), c, "-o", exe,
+                        "-L", libdir, "-lmala", "-Wl,-rpath," + libdir], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True)
+    assert out.returncode == 0, out.stdout + out.stderr
+    first, second = out.stdout.split("\n")[:2]
+    assert first.split()[1:] == ["MALA_ERR_TIMEOUT", str(mala.MALA_ERR_INVALID_ARG), "msg"]
+    assert second == "0"
