@@ -297,3 +297,28 @@ int main(void) {
     first, second = out.stdout.split("\n")[:2]
     assert first.split()[1:] == ["MALA_ERR_TIMEOUT", str(mala.MALA_ERR_INVALID_ARG), "msg"]
     assert second == "0"
+
+
+def test_decode_marshalling_fills_every_field(monkeypatch):
+    """The binding's decode struct, filled from host tensors with the CUDA
+    guard patched out (nothing is called): shapes, strides, element types,
+    scales and the group-voting flag reach the C struct."""
+    import torch
+    monkeypatch.setattr(mala, "_require_cuda", lambda *ts: None)
+    q = torch.zeros(3, 1, 8, 128, dtype=torch.bfloat16)
+    k = torch.zeros(3, 1000, 2, 128, dtype=torch.float8_e4m3fn)
+    o, lse, keep, a, keep_alive = mala._decode_call(q, k, k, 0.5, 128, 2, None, None, None, True, None, None,
+                                                    0.25, 4.0, True)
+    assert (a.batch, a.heads_q, a.heads_kv, a.seqlen_k, a.head_dim) == (3, 8, 2, 1000, 128)
+    assert list(a.k_stride) == [1000 * 2 * 128, 2 * 128, 128] and list(a.q_stride) == [8 * 128, 8 * 128, 128]
+    assert a.kv_dtype == mala.MALA_FP8_E4M3 and (a.k_scale, a.v_scale) == (0.25, 4.0)
+    assert a.group_vote == 1 and a.num_splits == 2 and a.block_k == 128 and a.tau == 0.5
+    assert a.dtype == mala.MALA_BF16
+    assert a.o == o.data_ptr() and a.lse == lse.data_ptr() and a.keep_mask == keep.data_ptr()
+    assert keep.shape == (3, 8, 1) and lse.shape == (3, 8)
+    kb = torch.zeros(3, 1000, 2, 128, dtype=torch.bfloat16)
+    _, _, keep2, a2, _ = mala._decode_call(q, kb, kb, 0.5, 128, 0, None, None, None, False, None, None,
+                                           1.0, 1.0, False)
+    assert a2.kv_dtype == mala.MALA_BF16 and a2.group_vote == 0 and keep2 is None and not a2.keep_mask
+    with pytest.raises(ValueError):
+        mala._decode_call(q, k, kb, 0.5, 128, 0, None, None, None, True, None, None, 1.0, 1.0, False)
