@@ -144,9 +144,17 @@ def whole_job_rate(units_per_rank: float, world: int, seconds: float) -> float:
     return units_per_rank * world / seconds
 
 
-def tile_flops(d: int = 128) -> float:
-    """FLOPs of one 128 x 128 x d tile matmul (2 per multiply-add)."""
-    return 2.0 * TILE * TILE * d
+def tile_flops(d: int = 128, bq: int = TILE, bk: int = TILE) -> float:
+    """FLOPs of one bq x bk x d tile matmul (2 per multiply-add)."""
+    return 2.0 * bq * bk * d
+
+
+def tc_fracs(tflops: float, peaks) -> dict:
+    """Fractions of the measured dense bf16 peak: the burst figure (cuBLAS
+    timed alone, the headline denominator) and the sustained one (cuBLAS
+    looped for seconds under the power cap)."""
+    return {"frac_of_peak": tflops / peaks["bf16_tflops"],
+            "frac_of_sustained": tflops / peaks["bf16_tflops_sustained"]}
 
 
 def run_mala(args):
@@ -346,11 +354,12 @@ def run_mala(args):
     grp = None if args.no_extras else bench_group_fwd(args, q, k, v, stream, peaks)
     dec = None if args.no_decode else bench_decode(args, dev, stream, peaks)
     dec8 = None if args.no_decode else bench_decode(args, dev, stream, peaks, e4m3=True)
+    cfgs = None if args.no_configs else bench_configs(args, dev, stream, peaks)
     kern_f = statistics.mean(fwd_times)
     kern_b = statistics.mean(bwd_times)
     ach_f = fwd_flops / kern_f / 1e12
     ach_b = bwd_flops / kern_b / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    peak = peaks["bf16_tflops"]
     dom = ("mala_bwd (pre + mala_bwd_tc_kernel + dQ conversion)", ach_b) if kern_b >= kern_f \
         else ("mala_fwd_tc_kernel<128>", ach_f)
     res = {
@@ -370,10 +379,10 @@ def run_mala(args):
                    "head_dim": d, "block_q": TILE, "block_k": TILE, "tau": TAU, "pass": "fwd+bwd",
                    "l2": "inputs (0.7 GB) larger than L2; no flush"},
         "tflops_executed": (fwd_flops + bwd_flops) / (elapsed / args.steps / world) / 1e12,
-        "fwd": {"ms": kern_f * 1e3, "tflops_executed": ach_f, "frac_of_peak": ach_f / peak,
+        "fwd": {"ms": kern_f * 1e3, "tflops_executed": ach_f, **tc_fracs(ach_f, peaks),
                 "tiles_tested": tested, "tiles_kept": kept, "kept_fraction": kept / tested,
                 "slots_per_query": slots / (B * Hq * N)},
-        "bwd": {"ms": kern_b * 1e3, "tflops_executed": ach_b, "frac_of_peak": ach_b / peak,
+        "bwd": {"ms": kern_b * 1e3, "tflops_executed": ach_b, **tc_fracs(ach_b, peaks),
                 "tiles_visited": b_visit, "tiles_kept": b_kept, "kept_fraction": b_kept / max(b_visit, 1),
                 "slots_per_query": b_slots / (B * Hq * N)},
         "tau0": {"ms_per_step": dense_s * 1e3, "tokens_per_s": whole_job_rate(B * N, world, dense_s),
@@ -384,7 +393,8 @@ def run_mala(args):
         "tau_sweep": sweep,
         "roofline": {"bound": "tensor", "kernel": dom[0], "achieved": dom[1],
                      "peak": peak, "unit": "TFLOP/s", "frac": dom[1] / peak,
-                     "peak_source": f"{peaks['source']} bf16_tflops_sustained",
+                     "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                     "frac_of_sustained": dom[1] / peaks["bf16_tflops_sustained"],
                      "traffic": (NCU_TRAFFIC.get("mala_bwd_tc_kernel")
                                  if kern_b >= kern_f and N == 32768 else None),
                      "traffic_note": "ncu DRAM bytes of the mala_bwd_tc_kernel launch (bytes per launch)"},
@@ -399,6 +409,8 @@ def run_mala(args):
     if dec is not None:
         res["decode"] = dec
         res["decode_e4m3"] = dec8
+    if cfgs is not None:
+        res["configs"] = cfgs
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
     if world > 1:
@@ -436,10 +448,9 @@ def bench_chunk(args, q, k, v, stream, peaks, chunk: int = 4096):
     mala.check_device_error()
     t = e0.elapsed_time(e1) / 1e3 / n
     flops = tile_flops(q.shape[3]) * (tested + kept)
-    peak = peaks["bf16_tflops_sustained"]
     return {"seqlen_q": chunk, "seqlen_k": Nk, "tau": TAU, "ms": t * 1e3,
             "tokens_per_s": q.shape[0] * chunk / t, "tiles_tested": tested, "tiles_kept": kept,
-            "tflops_executed": flops / t / 1e12, "frac_of_peak": flops / t / 1e12 / peak}
+            "tflops_executed": flops / t / 1e12, **tc_fracs(flops / t / 1e12, peaks)}
 
 
 def bench_group_fwd(args, q, k, v, stream, peaks, taus=(TAU, 64.0)):
@@ -477,12 +488,13 @@ def bench_group_fwd(args, q, k, v, stream, peaks, taus=(TAU, 64.0)):
             flops = tile_flops(d) * (tested + kept)
             row[mode] = {"ms": t * 1e3, "tiles_tested": tested, "tiles_kept": kept,
                          "kept_fraction": kept / tested, "tflops_executed": flops / t / 1e12,
-                         "frac_of_peak": flops / t / 1e12 / peaks["bf16_tflops_sustained"]}
+                         **tc_fracs(flops / t / 1e12, peaks)}
         out[str(tau)] = row
     return out
 
 
-def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072, e4m3: bool = False):
+def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072, e4m3: bool = False,
+                 with_group: bool = True):
     """Split-KV decode on the largest decode workload (batch 64, 32 query
     heads, 8 KV heads, d = 128, bf16 cache of seqlen_k keys, tau = 0.05).
     The 34 GB cache is drawn on the device with the decode recipe (sink key,
@@ -493,7 +505,7 @@ def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072, e4m3: bool = 
     import torch
     from tile_skipping_causal_b200 import mala, synth
 
-    w = synth.decode_workload(args.decode_seqlen or seqlen_k)
+    w = synth.decode_workload(seqlen_k if args.decode_seqlen is None or seqlen_k != 131072 else args.decode_seqlen)
     q = synth.make_decode_query(w, SEED).to(dev)
     k, v = synth.fill_decode_cache(w, SEED, q.cpu(), dev, slices=[])
     if e4m3:
@@ -526,7 +538,7 @@ def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072, e4m3: bool = 
     mala.check_device_error()
     t = e0.elapsed_time(e1) / 1e3 / n
     group = None
-    if not e4m3:
+    if with_group and not e4m3:
         # group-joint voting (one decision per key tile for the query heads of
         # a KV head) on the same cache
         gstats = torch.zeros(4, dtype=torch.int64, device=dev)
@@ -566,6 +578,110 @@ def bench_decode(args, dev, stream, peaks, seqlen_k: int = 131072, e4m3: bool = 
                          "traffic": NCU_TRAFFIC.get(f"mala_decode_split_kernel@{w.seqlen_k}" + ("/e4m3" if e4m3 else "")),
                          "traffic_note": "ncu DRAM bytes per launch, N_k = 8192 capture scaled by N_k"},
             "group_vote": group}
+
+
+L2_FLUSH_BYTES = 256 << 20          # twice the 126 MB L2
+
+
+def _time_flushed(fn, n: int, stream, flush) -> float:
+    """Mean device time of ``fn`` over n calls, each preceded (outside its
+    own CUDA events) by a write of a buffer larger than L2, so that no call
+    finds the previous call's inputs in L2."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+
+
+def bench_configs(args, dev, stream, peaks) -> dict:
+    """Every benchmark configuration of the operator at its own taus, each
+    beside tau = 0 (FullAttn) on the same inputs and kernels: device time,
+    tokens/s, executed TFLOP/s (every tested tile pays QK^T, every retained
+    one PV; the backward pays the recomputed S^T per visited tile and four
+    matmuls per retained one), kept-tile fractions and post-score key slots
+    per query (the pages' cost measure). Each timed call starts with L2
+    flushed. Decoding: the decode workload at every cache length with its
+    HBM roofline (the largest length is the separate "decode" entry)."""
+    import torch
+    from tile_skipping_causal_b200 import mala, synth
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    n = max(5, args.steps // 2)
+    out = {}
+
+    def prefill(name, taus, backward):
+        w = synth.WORKLOADS[name]
+        t = {k_: x.to(dev) for k_, x in synth.make_prefill(w, SEED, with_do=backward).items()}
+        q, k, v = t["q"], t["k"], t["v"]
+        B, N, Hq, d = q.shape
+        fp32 = w.dtype == "fp32"
+        bq, bk = w.block_q, w.block_k
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+        nKB = -(-N // bk)
+        keep = torch.empty((B, Hq, -(-N // bq), mala.mask_words(nKB)), dtype=torch.int32, device=dev)
+        if backward:
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        rows = []
+        for tau in (0.0,) + tuple(taus):
+            st = torch.zeros(4, dtype=torch.int64, device=dev)
+            bst = torch.zeros(4, dtype=torch.int64, device=dev)
+            mala.mala_fwd(q, k, v, tau, bq, bk, o=o, lse=lse, keep_mask=keep, stats=st)
+            if backward:
+                mala.mala_bwd(q, k, v, o, t["do"], lse, tau, keep, dq=dq, dk=dk, dv=dv, stats=bst)
+            mala.check_device_error()
+            tested, kept, slots = (int(x) for x in st.cpu().tolist()[:3])
+            fwd = lambda: mala.mala_fwd(q, k, v, tau, bq, bk, o=o, lse=lse, keep_mask=keep)
+            for _ in range(3):
+                fwd()
+            tf = _time_flushed(fwd, n, stream, flush)
+            ff = tile_flops(d, bq, bk) * (tested + kept)
+            row = {"tau": tau, "fwd_ms": tf * 1e3, "fwd_tflops_executed": ff / tf / 1e12,
+                   "fwd_tiles_tested": tested, "fwd_tiles_kept": kept, "fwd_kept_fraction": kept / tested,
+                   "fwd_slots_per_query": slots / (B * Hq * N)}
+            if not fp32:
+                row.update({"fwd_" + k_: x for k_, x in tc_fracs(ff / tf / 1e12, peaks).items()})
+            total = tf
+            if backward:
+                bv, bkp, bsl = (int(x) for x in bst.cpu().tolist()[:3])
+                bwd = lambda: mala.mala_bwd(q, k, v, o, t["do"], lse, tau, keep, dq=dq, dk=dk, dv=dv)
+                for _ in range(3):
+                    bwd()
+                tb = _time_flushed(bwd, n, stream, flush)
+                bf = tile_flops(d) * (bv + 4 * bkp)
+                row.update({"bwd_ms": tb * 1e3, "bwd_tflops_executed": bf / tb / 1e12,
+                            "bwd_tiles_visited": bv, "bwd_tiles_kept": bkp,
+                            "bwd_kept_fraction": bkp / max(bv, 1), "bwd_slots_per_query": bsl / (B * Hq * N)})
+                row.update({"bwd_" + k_: x for k_, x in tc_fracs(bf / tb / 1e12, peaks).items()})
+                total += tb
+            mala.check_device_error()
+            row["tokens_per_s"] = B * N / total
+            rows.append(row)
+        dense_ms = rows[0]["fwd_ms"] + rows[0].get("bwd_ms", 0.0)
+        for r in rows:
+            r["speedup_vs_tau0"] = dense_ms / (r["fwd_ms"] + r.get("bwd_ms", 0.0))
+        out[name] = {"batch": B, "heads_q": Hq, "heads_kv": k.shape[2], "seqlen": N, "head_dim": d,
+                     "block_q": bq, "block_k": bk, "dtype": w.dtype,
+                     "pass": "fwd+bwd" if backward else "fwd", "per_tau": rows}
+        if fp32:
+            out[name]["note"] = "fp32 CUDA-core path (64 x 64 tiles); inputs fit in L2, which is flushed"
+        del t, q, k, v, o
+        torch.cuda.empty_cache()
+
+    prefill("toy_fp32_512", synth.WORKLOADS["toy_fp32_512"].taus, False)
+    prefill("prefill_4k", synth.WORKLOADS["prefill_4k"].taus, False)
+    prefill("train_8k", synth.WORKLOADS["train_8k"].taus, True)
+    del flush
+    torch.cuda.empty_cache()
+    if not args.no_decode:
+        out["decode_sweep"] = [bench_decode(args, dev, stream, peaks, seqlen_k=nk, with_group=False)
+                               for nk in synth.DECODE_SEQLENS if nk != 131072]
+    return out
 
 
 _ORACLE_INPUTS = {}
@@ -675,6 +791,10 @@ def main():
                     help="run only the decode measurement (profiling captures)")
     ap.add_argument("--decode-e4m3", action="store_true",
                     help="with --decode-only: an e4m3 cache instead of bf16")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration measurements (prefill_4k, train_8k, decode sweep, toy)")
+    ap.add_argument("--configs-only", action="store_true",
+                    help="run only the per-configuration measurements")
     ap.add_argument("--group-only", action="store_true",
                     help="run only the group-joint voting forward measurement")
     ap.add_argument("--no-extras", action="store_true",
@@ -692,6 +812,13 @@ def main():
         t = synth.make_prefill(synth.WORKLOADS[WORKLOAD], SEED, seqlen=args.seqlen)
         q, k, v = (t[n].to(dev) for n in ("q", "k", "v"))
         print(json.dumps(bench_group_fwd(args, q, k, v, torch.cuda.current_stream(), _peaks())), flush=True)
+    elif args.configs_only:
+        import torch
+        from tile_skipping_causal_b200 import mala
+        mala.load_library()
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps(bench_configs(args, dev, torch.cuda.current_stream(), _peaks())), flush=True)
     elif args.decode_only:
         import torch
         from tile_skipping_causal_b200 import mala

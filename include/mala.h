@@ -283,7 +283,10 @@ MALA_API int mala_decode(mala_decode_args* args, void* workspace, size_t workspa
  *     MALA_ERR_WORKSPACE with the sizes in mala_last_error_message().
  *   - The first call on each device looks up the buffer's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture. The address is kept for the life of the
+ *     process: after cudaDeviceReset() on a device, do not call this entry
+ *     point on that device again in the same process (the library's device
+ *     error block, looked up the same way, has the same limit).
  *   - All calls share the one buffer, which keeps the last call's contents.
  *     Calls whose kernels overlap on the GPU (e.g. on different streams
  *     without ordering) race on it and give wrong results: order them.

@@ -110,7 +110,23 @@ def test_pure_backward_equals_mask_replay_and_nests():
     fm = mala.unpack_mask(keep, 6)
     b1 = mala.unpack_mask(bkeep, 6)
     b2 = mala.unpack_mask(bkeep2, 6)
-    assert not (b2 & ~fm).any() or (b2 & ~fm).sum() <= 2
+    # Support nesting ("Offline Sparse Probability"): a tile the pure
+    # backward retains was retained by the forward, up to rounding. Each
+    # exception must be a near-tie: the oracle's forward margin or its pure
+    # backward margin for that tile lies within the 1e-3-nat band.
+    viol = np.argwhere(b2 & ~fm)
+    if len(viol):
+        from tests.parity import MARGIN_BAND, as_operator_outputs, f64
+        q64, k64, v64, do64 = (f64(t[n]) for n in ("q", "k", "v", "do"))
+        G = q64.shape[2] // k64.shape[2]
+        for (b, h, i, j) in viol:
+            Q, K, V = q64[b, :, h], k64[b, :, h // G], v64[b, :, h // G]
+            O, z, _, fmarg = orc.forward_head(Q, K, V, 128, 128, 0.1)
+            Ob, zf = as_operator_outputs(O, z)
+            _, _, _, _, bmarg = orc.backward_head(Q, K, V, Ob, do64[b, :, h], zf, 128, 128, 0.1, None)
+            near = min(abs(fmarg[i, j]), abs(bmarg[i, j]))
+            assert near <= MARGIN_BAND, f"tile ({b},{h},{i},{j}) breaks nesting with margins " \
+                                        f"{fmarg[i, j]:.3e} (fwd) / {bmarg[i, j]:.3e} (bwd)"
     assert (b1 == (b2 & fm)).all()
     for a, c in ((dq, dq2), (dk, dk2), (dv, dv2)):
         assert torch.equal(a, c) or (a.float() - c.float()).norm() <= 1e-2 * c.float().norm()
@@ -151,6 +167,43 @@ def test_train_8k_full_size_sampled():
     fm = mala.unpack_mask(keep, nQB)
     bm = mala.unpack_mask(bkeep, nQB)
     assert s[0] == fm.sum() and s[1] == bm.sum()
+
+
+@pytest.fixture(scope="module")
+def gqa32k_do():
+    return _run(synth.WORKLOADS["gqa_32k"])
+
+
+@pytest.mark.parametrize("tau", [0.2, 64.0])
+def test_gqa_32k_full_size_fwd_bwd_sampled(gqa32k_do, tau):
+    """The benchmark's step at its own size (batch 1, 32 query heads, 8 KV
+    heads, N = 32768): forward then mask-replay backward in the launch
+    configuration the benchmark times, at the workload's tau and at tau = 64,
+    where this data skips tiles in both passes. Sampled against the oracle:
+    forward query blocks and dQ rows from each head third (diffuse 0-10,
+    local 11-21, retrieval 22-31), and dK/dV of key blocks of one KV head from
+    each third (every query head of the group, every query block that sees
+    the key block)."""
+    from tests.parity import check_fwd
+    t = gqa32k_do
+    stats = torch.zeros(4, dtype=torch.int64, device=DEV)
+    bstats = torch.zeros(4, dtype=torch.int64, device=DEV)
+    o, lse, keep = mala.mala_fwd(t["q"], t["k"], t["v"], tau, 128, 128, stats=stats)
+    dq, dk, dv, bkeep = mala.mala_bwd(t["q"], t["k"], t["v"], o, t["do"], lse, tau, keep,
+                                      with_bwd_mask=True, stats=bstats)
+    mala.check_device_error()
+    fs, bs = stats.cpu().tolist(), bstats.cpu().tolist()
+    assert fs[0] == 32 * 256 * 257 // 2
+    if tau == 64.0:
+        assert fs[1] < 0.9 * fs[0] and bs[1] < 0.9 * bs[0]     # both passes skip
+    fsamples = [(0, h, i) for h in (2, 16, 29) for i in (0, 131, 255)]
+    rep = check_fwd(t["q"], t["k"], t["v"], o, lse, keep, tau, 128, 128, fsamples)
+    assert rep.blocks == len(fsamples)
+    kv = [(0, 0, 255), (0, 3, 200), (0, 6, 120), (0, 7, 253)]
+    qs = [(0, 0, 0), (0, 13, 100), (0, 24, 255), (0, 31, 180)]
+    brep = check_bwd_blocks(t["q"], t["k"], t["v"], t["do"], keep, bkeep, dq, dk, dv, tau,
+                            kv_samples=kv, q_samples=qs)
+    assert brep["worst_rel_fro"] < 3e-2
 
 
 # ------------------------------------------- bottom-right causal alignment

@@ -61,6 +61,32 @@ def test_decode_full_size_sampled(Nk):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("Nk,splits,tau", [(1000, 1, 5.0), (1000, 3, 50.0), (4096, 0, 5.0),
+                                           (4096, 1, 50.0), (4096, 3, 50.0), (129, 0, 50.0)])
+def test_decode_per_head_with_disagreeing_group_heads(Nk, splits, tau):
+    """Per-head decisions ("Fused decoding execution"): a V tile is read when
+    some head of the group retains it, and only the retaining heads
+    accumulate it. At these tau the needle recipe makes heads of one group
+    disagree on many tiles, so the kernel runs the path that loads V for the
+    group and zeroes P for the heads that skip."""
+    w, q, k, v = _small(2, Nk, seed=21)
+    stats = torch.zeros(4, dtype=torch.int64, device=DEV)
+    o, lse, keep, P = _decode(q, k, v, tau, splits, stats=stats)
+    if splits:
+        assert P == splits
+    nKB = -(-Nk // 128)
+    m = mala.unpack_mask(keep, nKB).reshape(2, 8, 4, nKB)
+    disagree = m.any(axis=2) & ~m.all(axis=2)
+    if Nk >= 1000:
+        assert disagree.sum() > 0, "no tile with heads of one group deciding differently"
+    tested, vread, kept_heads = (int(x) for x in stats.cpu().tolist()[:3])
+    assert tested == 2 * 8 * nKB
+    assert vread == int(m.any(axis=2).sum())          # V read iff some head of the group retains
+    assert kept_heads == int(m.sum())
+    rep = check_decode(q, k, v, o, lse, keep, tau, P)
+    assert rep.heads == 2 * 32
+
+
 def test_decode_tau_zero_is_dense():
     w, q, k, v = _small(1, 777)
     o, lse, keep, P = _decode(q, k, v, 0.0, 2)
@@ -139,6 +165,19 @@ def test_decode_e4m3_cache(Nk, splits, scales):
     rep = check_decode(q, kd, vd, o, lse, keep, w.tau, P)
     assert rep.heads == 2 * 32
     assert stats[0].item() == 2 * 8 * -(-Nk // 128)
+
+
+def test_decode_e4m3_per_head_with_disagreeing_group_heads():
+    """The e4m3 instantiation of the per-head path at a tau where heads of a
+    group disagree (V read for the group, P zeroed for skipping heads)."""
+    w, q, k, v = _small(2, 3000, seed=22)
+    kc, kd = _quantise(k, 0.5)
+    vc, vd = _quantise(v, 1.5)
+    o, lse, keep, P = _decode(q, kc, vc, 50.0, 0, k_scale=0.5, v_scale=1.5)
+    m = mala.unpack_mask(keep, 24).reshape(2, 8, 4, 24)
+    assert (m.any(axis=2) & ~m.all(axis=2)).sum() > 0
+    rep = check_decode(q, kd, vd, o, lse, keep, 50.0, P)
+    assert rep.heads == 2 * 32
 
 
 def test_decode_e4m3_large_cache_sampled():

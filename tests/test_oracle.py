@@ -405,6 +405,74 @@ def test_decode_first_tile_of_each_split_retained():
     assert orc.split_ranges(10, 3) == [(0, 3), (3, 6), (6, 10)]
 
 
+def _brute_decode_row(q, K, V, Bk, tau, P):
+    """One decoding query in ratio form with explicit retained key sets, per
+    split: walking a split's tiles from the last, a tile is retained iff the
+    split's retained set is empty or some key of the tile has
+    exp(s) / sum over retained keys of exp(s) >= tau / N_k. Each split's
+    partial is plain softmax attention over its retained keys; the split
+    results combine as sum_p Z_p O_p / sum_p Z_p (Z_p = sum of exp(s) over
+    split p's retained keys). Returns O, log sum_p Z_p, keep."""
+    N = K.shape[0]
+    s = K @ q
+    nKB = -(-N // Bk)
+    keep = np.zeros(nKB, dtype=bool)
+    num = np.zeros(V.shape[1])
+    den = 0.0
+    for (t0, t1) in orc.split_ranges(nKB, P):
+        kept_keys = []
+        for j in range(t1 - 1, t0 - 1, -1):
+            keys = list(range(j * Bk, min((j + 1) * Bk, N)))
+            if kept_keys:
+                ratio = math.exp(max(s[keys])) / sum(math.exp(s[k]) for k in kept_keys)
+                keep[j] = not (ratio < tau / N)
+            else:
+                keep[j] = True
+            if keep[j]:
+                kept_keys += keys
+        w = np.array([math.exp(s[k]) for k in kept_keys])
+        num += w @ V[kept_keys]
+        den += w.sum()
+    return num / den, math.log(den), keep
+
+
+@pytest.mark.parametrize("P,tau", [(1, 0.0), (2, 0.5), (3, 4.0)])
+def test_decode_batched_gqa_head_mapping(P, tau):
+    """oracle.decode over [B, 1, H_q, d] queries and a [B, N_k, H_kv, d]
+    cache: query head h of batch b reads KV head h // (H_q / H_kv) of the same
+    batch. Every (b, h) is checked against the brute-force ratio form run on
+    that KV head's rows; at tau = 0 also against torch's dense softmax with
+    the KV heads repeated G times along the head axis (the usual GQA
+    expansion). The cache's KV heads and batches differ, so a transposed
+    head map or batch index fails."""
+    rng = np.random.default_rng(200 + P)
+    B, Hq, Hkv, N, d, Bk = 2, 8, 2, 45, 6, 8
+    G = Hq // Hkv
+    q = rng.standard_normal((B, 1, Hq, d)) * 4 / math.sqrt(d)
+    k = rng.standard_normal((B, N, Hkv, d))
+    v = rng.standard_normal((B, N, Hkv, d))
+    O, lse, keep, _ = orc.decode(q, k, v, Bk, tau, P)
+    for b in range(B):
+        for h in range(Hq):
+            Ob, zb, kb = _brute_decode_row(q[b, 0, h], k[b, :, h // G], v[b, :, h // G], Bk, tau, P)
+            assert (keep[b, h] == kb).all(), (b, h)
+            assert np.allclose(O[b, 0, h], Ob, atol=1e-12), (b, h)
+            assert abs(lse[b, h] - zb) < 1e-12, (b, h)
+            # another KV head gives other values: the map is observable here
+            Ow, _, _ = _brute_decode_row(q[b, 0, h], k[b, :, 1 - h // G], v[b, :, 1 - h // G], Bk, tau, P)
+            assert not np.allclose(O[b, 0, h], Ow, atol=1e-6)
+    if tau == 0.0:
+        qt = torch.tensor(q)
+        ke = torch.tensor(k).repeat_interleave(G, dim=2)
+        ve = torch.tensor(v).repeat_interleave(G, dim=2)
+        s = torch.einsum("bqhd,bkhd->bhqk", qt, ke)
+        out = torch.einsum("bhqk,bkhd->bqhd", torch.softmax(s, -1), ve)
+        assert np.abs(O - out.numpy()).max() < 1e-12
+        assert np.abs(lse - torch.logsumexp(s, -1)[:, :, 0].numpy()).max() < 1e-12
+    else:
+        assert not keep.all()                        # the case skips tiles
+
+
 def _group_case(seed, G, N, d, sharp=3.0):
     rng = np.random.default_rng(seed)
     Qg = rng.standard_normal((G, d)) * sharp / math.sqrt(d)

@@ -31,11 +31,11 @@ def _lib():
     mala.load_library()
 
 
-def _inputs(seed, Nk=4096):
+def _inputs(seed, Nk=4096, Hkv=8):
     # decode workload shape with the sink / needle recipe: batch 64, 32 query
     # heads, 8 KV heads; the library picks 3 splits, whose partials (3.2 MB)
     # fit in the built-in 4 MiB buffer
-    w = synth.DecodeWorkload("decode_noalloc", 64, 32, 8, Nk, 128, 128, 0.05)
+    w = synth.DecodeWorkload("decode_noalloc", 64, 32, Hkv, Nk, 128, 128, 0.05)
     q = synth.make_decode_query(w, seed)
     k, v = synth.fill_decode_cache(w, seed, q, DEV, slices=[])
     return w, q.to(DEV), k, v
@@ -68,4 +68,23 @@ def test_noalloc_rejects_partials_larger_than_the_buffer():
     mala.check_device_error()
     assert p == fits
     assert_close(f64(o), f64(o_ref), "O", ATOL, RTOL)
+    assert torch.equal(keep, keep_ref)
+
+
+def test_noalloc_lowers_the_automatic_split_count_to_fit():
+    """With 4 KV heads per sequence the automatic choice is 5 splits, whose
+    partials (5.3 MB) exceed the built-in buffer; the entry point lowers the
+    count until they fit (3 splits, 3.2 MB) and then computes what the
+    workspace entry point computes with that many splits."""
+    w, q, k, v = _inputs(14, Nk=4096, Hkv=4)
+    per_split = w.batch * w.heads_q * (128 + 1) * 4
+    _, _, _, p_auto = mala.mala_decode(q, k, v, w.tau, 128, 0)
+    o, lse, keep, p = mala.mala_decode_noalloc(q, k, v, w.tau, 128, 0)
+    mala.check_device_error()
+    assert per_split * p_auto > mala.DECODE_NOALLOC_SCRATCH_BYTES
+    assert 1 < p < p_auto and per_split * p <= mala.DECODE_NOALLOC_SCRATCH_BYTES < per_split * (p + 1)
+    o_ref, lse_ref, keep_ref, p_ref = mala.mala_decode(q, k, v, w.tau, 128, p)
+    assert p_ref == p
+    assert_close(f64(o), f64(o_ref), "O", ATOL, RTOL)
+    assert_close(lse.cpu().numpy(), lse_ref.cpu().numpy(), "LSE", ATOL, RTOL)
     assert torch.equal(keep, keep_ref)
