@@ -14,9 +14,9 @@
 //
 // Roles (320 threads): warps 0-7 compute in two warpgroups that split the
 // 128 query columns of a tile (lane t of TMEM is key row t for S^T, P^T,
-// dP^T, dS^T and query row t for the dQ part), warp 8 TMA producer
-// (in order, blocking waits: Q of the next tiles and dO of retained tiles), warp 9 tcgen05
-// issuer.
+// dP^T, dS^T and query row t for the dQ part), warp 8 TMA producer (in
+// order, blocking waits: Q of the next tiles, dO one tile ahead), warp 9
+// tcgen05 issuer.
 // TMEM: X = cols [0,128): S^T(n), then P^T(n) as packed bf16 in [0,64),
 // read by the dV MMA straight from TMEM; Y = [128,256): dP^T(n), then the
 // tile's dQ part; dK = [256,384); dV = [384,512).
@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
   if (tid == 0) {
     for (int x = 0; x < kNumBars; ++x) {
       uint32_t cnt = 1;
-      if (x == kXRead || x == kPtFull || x == kDsFull || x == kYFree) cnt = 256;
+      if (x == kXRead || x == kPtFull || x == kDsFull || x == kYFree) cnt = 8;   // one per compute warp
       if (x == kQEmpty || x == kQEmpty + 1 || x == kDecEmpty) cnt = 2;
       mbar_init(&bars[x], cnt);
     }
@@ -191,36 +191,53 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         bulk_load(sst + 256, p.Dv + row0, 512, &bars[kQFull + st]);
         return true;
       };
-      // In order, with blocking waits: per tile n, read its decision (and
-      // load its dO when retained), then refill its Q stage with tile n + 2
-      // once tile n released it. Every wait is for the next event this role
-      // needs, so the thread sleeps in the barrier wait instead of polling.
+      // In order, with blocking waits. dO of tile n + 1 is loaded one tile
+      // ahead, before tile n + 1 is decided, into the single dO buffer as
+      // soon as tile n has finished with it (after dP^T(n) for a retained
+      // tile n, once its own load has landed for a skipped one), so that
+      // its latency stays off the path to dV. Per tile n: read its
+      // decision, refill the dO buffer, then refill tile n's Q stage with
+      // tile n + 2 once tile n released it. Every wait is for the next event
+      // this role needs, so the thread sleeps in the barrier wait instead
+      // of polling.
+      auto load_do = [&](int n) {
+        mbar_expect_tx(&bars[kDoFull], kTile);
+        for (int c = 0; c < 2; ++c)
+          tma_load_4d(sDO + c * kChunk, &p.tm_do, &bars[kDoFull], c * 64, info_h[n & 3],
+                      qrow0 + info_i[n & 3] * kB, tb);
+      };
       int n_total = -1;                         // number of tiles, once known
       for (int n = 0; n < 2 && n_total < 0; ++n)
         if (!load_q(n)) n_total = n;
-      int kc_load = 0;
+      if (n_total != 0) load_do(0);
+      int kept_seen = 0;                        // retained tiles before tile n
       bool ok = true;
       for (int n = 0; n_total < 0 || n < n_total; ++n) {
         ok = mbar_wait(&bars[kDecFull], n & 1, abort_flag, p.err, wait_tag(1, kDecFull, n));
         if (!ok) break;
         const uint32_t keep = misc[5];
         mbar_arrive(&bars[kDecEmpty]);
-        if (keep) {
-          ok = mbar_wait(&bars[kDoEmpty], (kc_load & 1) ^ 1, abort_flag, p.err, wait_tag(1, kDoEmpty, kc_load));
+        // tile n + 1 exists iff Q(n + 1) was not the end marker
+        if (n_total < 0 || n + 1 < n_total) {
+          if (keep)   // the MMAs of tile n release the buffer after dP^T(n)
+            ok = mbar_wait(&bars[kDoEmpty], kept_seen & 1, abort_flag, p.err, wait_tag(1, kDoEmpty, n));
+          else        // nothing reads it: wait for tile n's own load to land
+            ok = mbar_wait(&bars[kDoFull], n & 1, abort_flag, p.err, wait_tag(1, kDoFull, n));
           if (!ok) break;
-          mbar_expect_tx(&bars[kDoFull], kTile);
-          for (int c = 0; c < 2; ++c)
-            tma_load_4d(sDO + c * kChunk, &p.tm_do, &bars[kDoFull], c * 64, info_h[n & 3],
-                        qrow0 + info_i[n & 3] * kB, tb);
-          ++kc_load;
+          load_do(n + 1);
         }
+        if (keep) ++kept_seen;
         if (n_total < 0) {
           ok = mbar_wait(&bars[kQEmpty + (n & 1)], (n >> 1) & 1, abort_flag, p.err, wait_tag(1, kQEmpty + (n & 1), n));
           if (!ok) break;
           if (!load_q(n + 2)) n_total = n + 2;
         }
-        misc[2] = (static_cast<uint32_t>(n) << 16) | (static_cast<uint32_t>(kc_load) & 0xffff);
+        misc[2] = (static_cast<uint32_t>(n) << 16) | (static_cast<uint32_t>(kept_seen) & 0xffff);
       }
+      // the last tile's dO load (no tile reads it when that tile was
+      // skipped) must land before the CTA's shared memory is released
+      if (ok && n_total > 0)
+        ok = mbar_wait(&bars[kDoFull], (n_total - 1) & 1, abort_flag, p.err, wait_tag(1, kDoFull, n_total - 1));
       if (!ok) drain_pause_ns(50000);   // let copies already issued land
     }
   } else if (warp == 9) {
@@ -256,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         const int st = n & 1, stn = (n + 1) & 1;
         if (keep) {
           if (!mbar_wait(&bars[kPtFull], kc & 1, abort_flag, p.err, wait_tag(2, kPtFull, kc))) { ok = false; break; }
-          if (!mbar_wait(&bars[kDoFull], kc & 1, abort_flag, p.err, wait_tag(2, kDoFull, kc))) { ok = false; break; }
+          if (!mbar_wait(&bars[kDoFull], n & 1, abort_flag, p.err, wait_tag(2, kDoFull, n))) { ok = false; break; }
           tc_fence_after();
           // dV += P^T dO: A = P^T from TMEM (8 columns per 16 queries), B = dO MN-major
 #pragma unroll
@@ -313,9 +330,11 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         misc[3] = (static_cast<uint32_t>(n) << 16) | (static_cast<uint32_t>(kc) & 0xffff);
         ++n;
       }
-      // every MMA issued above must have finished before TMEM is read or freed
+      // every MMA issued above must have finished before TMEM is read or
+      // freed: wait for that regardless of the abort flag (MMAs always
+      // complete), bounded in time
       umma_commit(&bars[kDone]);
-      mbar_wait(&bars[kDone], 0, abort_flag, p.err, wait_tag(2, kDone, 0));
+      mbar_wait_drain(&bars[kDone], 0);
     }
   } else {
     // ===================== compute warpgroups =====================
@@ -352,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       reg_fence(q0);
       reg_fence(q1);
       tc_fence_before();
-      mbar_arrive(&bars[kYFree]);
+      warp_arrive(&bars[kYFree]);
       float* dst = p.dq_acc + qblock_index(p.seq, p.Hq, p.nQB, b, pend_h, pend_i) * (kB * kD) + r * 4;
 #pragma unroll
       for (int u = 0; u < 8; ++u)
@@ -376,13 +395,15 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       const float4* zl2_4 = reinterpret_cast<const float4*>(sStats + st * 384 + c0);
       const float4* thr_4 = reinterpret_cast<const float4*>(sStats + st * 384 + 128 + c0);
       const float4* dv_4 = reinterpret_cast<const float4*>(sStats + st * 384 + 256 + c0);
-      // test over this half of the S^T row. Legal entries: query columns
-      // x >= lim (at or after the key's position); padded query rows carry
-      // an infinite threshold and never count
+      // test over this half of the S^T row: retain iff some legal entry has
+      // s - t2 >= 0 (t2 = z + log tau - log L_q of the entry's query
+      // column). Illegal entries (keys after the query's position, and key
+      // rows past N_k) only occur in tiles whose last key lies beyond the
+      // block's first query position; there they are set to -inf once, which
+      // keeps them out of the test (-inf - t2 is -inf or NaN, and fmaxf
+      // ignores NaN) and makes their P^T exactly 0. Padded query columns
+      // carry t2 = z log2 e = +inf and drop out the same way.
       const bool oks = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], n & 1, abort_flag, p.err, wait_tag(0, kSFull, n)));
-      // first legal column of this half for key row r: query column c is at
-      // position i * 128 + c + q_off and sees key j * 128 + r iff that is >= it
-      const int lim = (j * kB + r) - (i * kB + q_off) - c0;
       uint32_t sr[2][32];
       if (oks) {
         tc_fence_after();
@@ -395,7 +416,17 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       }
       reg_fence(sr[0]);
       reg_fence(sr[1]);
-      bool vote = false;
+      if (j * kB + kB - 1 > i * kB + q_off) {
+        // query column c0 + x is at position i * 128 + c0 + x + q_off and
+        // sees key j * 128 + r iff that is >= it: x >= lim
+        const int lim = (j * kB + r) - (i * kB + q_off) - c0;
+#pragma unroll
+        for (int x = 0; x < 64; ++x)
+          if (x < lim) sr[x >> 5][x & 31] = __float_as_uint(-INFINITY);
+      }
+      float mx[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
 #pragma unroll
       for (int x4 = 0; x4 < 16; ++x4) {
         const float4 tv = thr_4[x4];
@@ -403,9 +434,12 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int x = 4 * x4 + e;
-          vote |= (x >= lim) && (__uint_as_float(sr[x >> 5][x & 31]) >= th[e]);
+          mx[x & 7] = fmaxf(mx[x & 7], __uint_as_float(sr[x >> 5][x & 31]) - th[e]);
         }
       }
+      const float mall = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const bool vote = mall >= 0.0f;
       const bool keep = bar_or(1, 256, vote);
       if (tid == 0) {
         misc[4] = (static_cast<uint32_t>(n) << 16) | (static_cast<uint32_t>(kc) & 0xffff);
@@ -424,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       }
       if (!keep) {
         tc_fence_before();
-        mbar_arrive(&bars[kXRead]);
+        warp_arrive(&bars[kXRead]);
         if (tid == 0) mbar_arrive(&bars[kQEmpty + st]);
         ++sk;
         ++n;
@@ -432,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         continue;
       }
 
-      // P^T = exp2(S^T log2e - z log2e) on legal entries, as bf16 pairs: kept
+      // P^T = exp2(S^T log2e - z log2e) (0 on illegal entries), as bf16 pairs: kept
       // in registers for dS and written over S^T in X for the dV MMA. Both
       // halves finished reading S^T before the vote, so the packed P^T
       // columns [32 half, 32 half + 32) may overwrite either half's S^T.
@@ -445,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int x = 4 * x4 + e;
-          pv[e] = (x >= lim) ? ex2_approx(fmaf(__uint_as_float(sr[x >> 5][x & 31]), kLog2e, -zz[e])) : 0.0f;
+          pv[e] = ex2_approx(fmaf(__uint_as_float(sr[x >> 5][x & 31]), kLog2e, -zz[e]));
         }
         pp[2 * x4] = pack_bf16x2(pv[0], pv[1]);
         pp[2 * x4 + 1] = pack_bf16x2(pv[2], pv[3]);
@@ -454,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       tmem_st16(tX + lane_addr + half * 32 + 16, &pp[16]);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars[kPtFull]);
+      warp_arrive(&bars[kPtFull]);
 
       if (pending) drain();
 
@@ -495,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars[kDsFull]);
+      warp_arrive(&bars[kDsFull]);
       if (tid == 0) mbar_arrive(&bars[kQEmpty + st]);
       pending = true;
       pend_h = h;

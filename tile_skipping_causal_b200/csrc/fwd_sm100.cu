@@ -66,7 +66,7 @@ enum Bar {
   kVFull = 9,            // 4
   kVEmpty = 13,          // 4
   kSFull = 17,           // 3 (per S buffer)
-  kSDone = 20,           // 3 (per S buffer, 256 arrivals): both softmax groups are done
+  kSDone = 20,           // 3 (per S buffer, one arrival per softmax warp): both softmax groups are done
                          // with the buffer's tile (P written if retained, S read if skipped);
                          // one phase per use of the buffer, so its parity cannot alias
   kTileDone = 23,        // 3 (per S buffer, MMA commit once per tile after its PV, or
@@ -135,16 +135,25 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // ---- work item: query blocks with more key tiles first. b is the batch
-  // index, or the sequence of a packed call; qrow0 / krow0 are the sequence's
-  // first query / key row and tb its batch coordinate in the tensor maps.
+  // ---- work item. b is the batch index, or the sequence of a packed call;
+  // qrow0 / krow0 are the sequence's first query / key row and tb its batch
+  // coordinate in the tensor maps.
+  // Fixed lengths: the grid runs band by band, a band being the G query
+  // heads of one KV head of one batch entry (p.head_order lists them
+  // together) over all query blocks, blocks with more key tiles first and
+  // the G heads of a block side by side. The CTAs resident at any time then
+  // stream the K / V tiles of one or two KV heads, which stay in L2, and the
+  // heavy-first order inside each band keeps the tail of the grid light.
   int i, b, h, Nq, Nk, qrow0, krow0, tb;
   if (p.seq.n == 0) {
-    const int BH = p.B * p.Hq;
-    i = p.nQB - 1 - static_cast<int>(blockIdx.x) / BH;
-    const int bh = static_cast<int>(blockIdx.x) % BH;
-    b = bh / p.Hq;
-    h = bh % p.Hq;
+    const int x = static_cast<int>(blockIdx.x);
+    const int HQB = p.Hq * p.nQB;
+    const int GQB = p.group * p.nQB;
+    b = x / HQB;
+    const int band = (x % HQB) / GQB;
+    const int r = (x % HQB) % GQB;
+    i = p.nQB - 1 - r / p.group;
+    h = p.head_order[band * p.group + r % p.group];
     Nq = p.N;
     Nk = p.Nk;
     qrow0 = krow0 = 0;
@@ -172,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
   if (tid == 0) {
     for (int x = 0; x < kNumBars; ++x) {
       uint32_t cnt = 1;
-      if (x >= kSDone && x < kSDone + kNS) cnt = 256;
+      if (x >= kSDone && x < kSDone + kNS) cnt = 8;   // one per softmax warp
       if (x == kDecEmpty || x == kDecEmpty + 1) cnt = 2;
       mbar_init(&bars[x], cnt);
     }
@@ -319,9 +328,11 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
           if (!issue_qk(t + kNS)) { ok = false; break; }
         }
       }
-      // make sure every MMA issued above has finished before TMEM is freed
+      // every MMA issued above must have finished before TMEM is freed:
+      // wait for that regardless of the abort flag (MMAs always complete),
+      // bounded in time
       umma_commit(&bars[kMmaDone]);
-      mbar_wait(&bars[kMmaDone], 0, abort_flag, p.err, wait_tag(2, kMmaDone, 0));
+      mbar_wait_drain(&bars[kMmaDone], 0);
     }
   } else {
     // ===================== softmax warpgroups =====================
@@ -431,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       }
       if (!keep) {
         tc_fence_before();
-        mbar_arrive(&bars[kSDone + sb]);
+        warp_arrive(&bars[kSDone + sb]);
         prev_kept = false;
         continue;
       }
@@ -492,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       xsum[(par * 2 + g) * 128 + r] = ps;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars[kSDone + sb]);
+      warp_arrive(&bars[kSDone + sb]);
       prev_kept = true;
       ++kc;
     }
@@ -559,7 +570,8 @@ size_t fwd_tc_smem_bytes(int head_dim) {
 }
 
 // Group-joint voting: clusters of G consecutive CTAs, which the work-item
-// order makes the G query heads of one KV head on the same query block.
+// order makes the G query heads of one KV head on the same query block
+// (fixed lengths; packed sequences list a block's heads side by side too).
 template <int D>
 cudaError_t launch_fwd_tc_clustered(const FwdTcParams& p, unsigned grid, int smem, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};

@@ -38,9 +38,11 @@ struct FwdTcParams {
   int nQB, nKB, mask_words;
   float log2_tau;       // log2(tau): -inf for tau = 0, +inf for tau = inf
   uint8_t kv_of_q[kMaxHeads];
+  uint8_t head_order[kMaxHeads];   // query heads listed KV head by KV head
   SeqTable seq;         // packed sequences: nQB / nKB / mask_words are then maxima
-  int group_vote;       // group-joint voting: the G = Hq / Hkv CTAs of a query
-  int group;            // block's KV-head group form one cluster (G <= 8)
+  int group;            // G = Hq / Hkv
+  int group_vote;       // group-joint voting: the G CTAs of a query block's
+                        // KV-head group form one cluster (G <= 8)
 };
 
 cudaError_t launch_fwd_tc(const FwdTcParams& p, int head_dim, cudaStream_t stream);

@@ -275,6 +275,15 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
     mala::FwdTcParams p;
     memset(&p, 0, sizeof(p));
     if ((rc = head_map(a->q_to_kv, a->heads_q, a->heads_kv, p.kv_of_q))) return rc;
+    // query heads in KV-head order (a stable sort by KV head), so that the
+    // grid can run the heads that share K / V side by side
+    {
+      int pos = 0;
+      for (int64_t hk = 0; hk < a->heads_kv; ++hk)
+        for (int64_t h = 0; h < a->heads_q; ++h)
+          if (p.kv_of_q[h] == hk) p.head_order[pos++] = static_cast<uint8_t>(h);
+    }
+    p.group = static_cast<int>(a->heads_q / a->heads_kv);
     if (a->group_vote) {
       const int G = static_cast<int>(a->heads_q / a->heads_kv);
       if (G > 8) return fail(MALA_ERR_UNSUPPORTED, "group-joint voting supports groups of at most 8 query heads");
@@ -282,7 +291,6 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
         if (p.kv_of_q[h] != h / G)
           return fail(MALA_ERR_UNSUPPORTED, "group-joint voting needs the default head map (h -> h / G)");
       p.group_vote = 1;
-      p.group = G;
     }
     // packed sequences: one batch entry of total_q / total_k rows
     const int64_t mb = packed ? 1 : a->batch;

@@ -46,6 +46,18 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
       : "memory");
 }
 
+// One arrival per warp on `bar` (initialised with one arrival per arriving
+// warp), once every lane of the warp has reached this point. Arrivals on one
+// mbarrier word are processed one at a time, so 256 threads arriving
+// separately hold the barrier for about a thousand cycles; a warp-wide
+// __syncwarp, which orders the lanes' earlier memory operations before lane
+// 0's release-arrive, replaces 32 of them. Lanes that wrote tensor memory
+// execute tcgen05.fence::before_thread_sync first.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile(
       "{\n\t.reg .b64 st;\n\t"
@@ -139,6 +151,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
         return false;
       }
     }
+  }
+}
+
+// Wait for a phase that completes no matter what the other roles do (the
+// commit of MMAs already issued, copies already in flight), ignoring the
+// abort flag, so that nothing still writes shared or tensor memory when the
+// CTA releases it. Gives up after kWaitLimitNs; returns whether the phase
+// completed.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
   }
 }
 
