@@ -350,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
     bool prev_kept = false;
     uint32_t mask_word = 0;
     int kept_tiles = 0;
+    int pending = -1;                        // group voting: tile whose exchange wait is deferred
     const int mask_base = (p.seq.n == 0 ? (b * p.Hq + h) * p.nQB + i
                                         : h * p.seq.qb0[p.seq.n] + p.seq.qb0[b] + i) * p.mask_words;
     if (tid == 0 && p.keep_mask) {
@@ -407,19 +408,25 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       const bool vote = has_key && (l == 0.0f || rmax2 - (m2 + lg2_approx(l)) >= thr2);
       bool keep = bar_or(1, 256, vote);
       if (p.group_vote) {
-        // group-joint voting: send this block's vote to every CTA of the
-        // cluster, then OR the G votes of tile t. A slot of parity par is
-        // rewritten (tile t + 2) only after every peer has passed the tile
-        // t + 1 exchange, hence after this CTA read it.
-        if (tid == 0) {
-          const uint32_t slot = smem_u32(const_cast<uint32_t*>(&cvote[par * 8 + crank]));
-          const uint32_t cbar = smem_u32(&cbars[par]);
-          for (int rr = 0; rr < p.group; ++rr) {
-            st_cluster_u32(mapa_shared(slot, rr), keep ? 1u : 0u);
-            mbar_arrive_cluster(mapa_shared(cbar, rr));
-          }
+        // group-joint voting. A CTA sends its tile t vote only after its
+        // own wait for tile t - 1 has completed, so no arrival for tile
+        // t + 2 can land in the phase that still collects tile t, and no
+        // peer rewrites a vote slot before this CTA has read it. When this
+        // CTA's own vote already retains the tile, the OR is known and the
+        // wait moves to the next tile's exchange, off the critical path.
+        if (pending >= 0) {
+          mbar_wait<true>(&cbars[pending & 1], (pending >> 1) & 1, abort_flag, p.err,
+                          wait_tag(0, 0x40 + (pending & 1), pending));
+          pending = -1;
         }
-        if (mbar_wait<true>(&cbars[par], (t >> 1) & 1, abort_flag, p.err, wait_tag(0, 0x40 + par, t))) {
+        if (tid < p.group) {          // one lane per peer, in parallel
+          const uint32_t slot = smem_u32(const_cast<uint32_t*>(&cvote[par * 8 + crank]));
+          st_cluster_u32(mapa_shared(slot, tid), keep ? 1u : 0u);
+          mbar_arrive_cluster(mapa_shared(smem_u32(&cbars[par]), tid));
+        }
+        if (keep) {
+          pending = t;
+        } else if (mbar_wait<true>(&cbars[par], (t >> 1) & 1, abort_flag, p.err, wait_tag(0, 0x40 + par, t))) {
           bool any = false;
           for (int rr = 0; rr < p.group; ++rr) any = any || cvote[par * 8 + rr] != 0u;
           keep = any;
