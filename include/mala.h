@@ -35,7 +35,8 @@
  *   - keep masks are uint32 bit sets: bit (j % 32) of word j / 32 of the
  *     row for (b, h, i) is set iff tile (i, j) was retained.
  *   - Kernels never trap. A device-side bounded wait that gives up records
- *     MALA_ERR_TIMEOUT, which mala_check_device_error() reports.
+ *     MALA_ERR_TIMEOUT, which mala_check_device_error() reports; the wait
+ *     limit is 2 s unless the call sets wait_limit_ns.
  */
 #ifndef MALA_H_
 #define MALA_H_
@@ -137,6 +138,13 @@ typedef struct {
    * the default head map (q_to_kv NULL or h -> h / G) and G <= 8, else
    * MALA_ERR_UNSUPPORTED; other values MALA_ERR_INVALID_ARG. */
   int32_t group_vote;
+  /* Limit in nanoseconds of every device-side bounded wait of this call;
+   * 0 (the default) means 2 s, far above any legitimate wait. A smaller
+   * value exists for tests of the timeout path: a wait that runs out makes
+   * the call's kernels stop early, leave their outputs undefined and record
+   * MALA_ERR_TIMEOUT for mala_check_device_error(). Negative values:
+   * MALA_ERR_INVALID_ARG. */
+  int64_t wait_limit_ns;
 } mala_fwd_args;
 
 #define MALA_MAX_SEQS 128
@@ -195,6 +203,13 @@ typedef struct {
    * the masks use mala_fwd's packed layouts. */
   const int32_t* cu_seqlens_q;
   const int32_t* cu_seqlens_k;
+  /* Limit in nanoseconds of every device-side bounded wait of this call;
+   * 0 (the default) means 2 s, far above any legitimate wait. A smaller
+   * value exists for tests of the timeout path: a wait that runs out makes
+   * the call's kernels stop early, leave their outputs undefined and record
+   * MALA_ERR_TIMEOUT for mala_check_device_error(). Negative values:
+   * MALA_ERR_INVALID_ARG. */
+  int64_t wait_limit_ns;
 } mala_bwd_args;
 
 MALA_API size_t mala_bwd_workspace_size(const mala_bwd_args* args);
@@ -257,6 +272,13 @@ typedef struct {
    * accumulated by every head of the group. keep_mask bits are then equal
    * across a group. Other values: MALA_ERR_INVALID_ARG. */
   int32_t group_vote;
+  /* Limit in nanoseconds of every device-side bounded wait of this call;
+   * 0 (the default) means 2 s, far above any legitimate wait. A smaller
+   * value exists for tests of the timeout path: a wait that runs out makes
+   * the call's kernels stop early, leave their outputs undefined and record
+   * MALA_ERR_TIMEOUT for mala_check_device_error(). Negative values:
+   * MALA_ERR_INVALID_ARG. */
+  int64_t wait_limit_ns;
 } mala_decode_args;
 
 MALA_API size_t mala_decode_workspace_size(const mala_decode_args* args);

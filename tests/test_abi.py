@@ -111,6 +111,7 @@ def _fwd_args(**kw):
     (dict(block_q=48), mala.MALA_ERR_UNSUPPORTED),
     (dict(mode=mala.MALA_DECODE), mala.MALA_ERR_UNSUPPORTED),
     (dict(dtype=7), mala.MALA_ERR_INVALID_ARG),
+    (dict(wait_limit_ns=-1), mala.MALA_ERR_INVALID_ARG),
 ])
 def test_fwd_rejects_bad_arguments_without_launching(lib, kw, code):
     a = _fwd_args(**kw)
@@ -183,6 +184,26 @@ def test_packed_sequence_count_limit(lib):
     assert "128" in lib.mala_last_error_message().decode()
 
 
+def test_backward_rejects_a_negative_wait_limit(lib):
+    a = mala.BwdArgs()
+    fake = 0x10000
+    a.q = a.k = a.v = a.o = a.dout = a.lse = a.dq = a.dk = a.dv = fake
+    a.batch, a.heads_q, a.heads_kv = 2, 4, 2
+    a.seqlen_q = a.seqlen_k = 256
+    a.head_dim = 128
+    for s in ("q_stride", "o_stride", "do_stride", "dq_stride"):
+        setattr(a, s, mala._i64x3(256 * 4 * 128, 4 * 128, 128))
+    for s in ("k_stride", "v_stride", "dk_stride", "dv_stride"):
+        setattr(a, s, mala._i64x3(256 * 2 * 128, 2 * 128, 128))
+    a.block_q = a.block_k = 128
+    a.tau = 0.1
+    a.dtype = mala.MALA_BF16
+    a.wait_limit_ns = -1
+    assert lib.mala_bwd_workspace_size(ctypes.byref(a)) == 0
+    assert lib.mala_bwd(ctypes.byref(a), None, 0, None) == mala.MALA_ERR_INVALID_ARG
+    assert "wait_limit_ns" in lib.mala_last_error_message().decode()
+
+
 def test_backward_checks_packed_offsets_too(lib):
     a = mala.BwdArgs()
     fake = 0x10000
@@ -222,7 +243,7 @@ def _decode_args(**kw):
 
 @pytest.mark.parametrize("kw", [dict(group_vote=2), dict(group_vote=-1), dict(kv_dtype=5),
                                 dict(kv_dtype=mala.MALA_FP8_E4M3, k_scale=0.0, v_scale=1.0),
-                                dict(num_splits=9)])
+                                dict(num_splits=9), dict(wait_limit_ns=-5)])
 def test_decode_rejects_bad_arguments_without_launching(lib, kw):
     a = _decode_args(**kw)
     assert lib.mala_decode_workspace_size(ctypes.byref(a)) == 0

@@ -213,22 +213,22 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       int kept_seen = 0;                        // retained tiles before tile n
       bool ok = true;
       for (int n = 0; n_total < 0 || n < n_total; ++n) {
-        ok = mbar_wait(&bars[kDecFull], n & 1, abort_flag, p.err, wait_tag(1, kDecFull, n));
+        ok = mbar_wait(&bars[kDecFull], n & 1, abort_flag, p.err, wait_tag(1, kDecFull, n), p.wait_ns);
         if (!ok) break;
         const uint32_t keep = misc[5];
         mbar_arrive(&bars[kDecEmpty]);
         // tile n + 1 exists iff Q(n + 1) was not the end marker
         if (n_total < 0 || n + 1 < n_total) {
           if (keep)   // the MMAs of tile n release the buffer after dP^T(n)
-            ok = mbar_wait(&bars[kDoEmpty], kept_seen & 1, abort_flag, p.err, wait_tag(1, kDoEmpty, n));
+            ok = mbar_wait(&bars[kDoEmpty], kept_seen & 1, abort_flag, p.err, wait_tag(1, kDoEmpty, n), p.wait_ns);
           else        // nothing reads it: wait for tile n's own load to land
-            ok = mbar_wait(&bars[kDoFull], n & 1, abort_flag, p.err, wait_tag(1, kDoFull, n));
+            ok = mbar_wait(&bars[kDoFull], n & 1, abort_flag, p.err, wait_tag(1, kDoFull, n), p.wait_ns);
           if (!ok) break;
           load_do(n + 1);
         }
         if (keep) ++kept_seen;
         if (n_total < 0) {
-          ok = mbar_wait(&bars[kQEmpty + (n & 1)], (n >> 1) & 1, abort_flag, p.err, wait_tag(1, kQEmpty + (n & 1), n));
+          ok = mbar_wait(&bars[kQEmpty + (n & 1)], (n >> 1) & 1, abort_flag, p.err, wait_tag(1, kQEmpty + (n & 1), n), p.wait_ns);
           if (!ok) break;
           if (!load_q(n + 2)) n_total = n + 2;
         }
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       // the last tile's dO load (no tile reads it when that tile was
       // skipped) must land before the CTA's shared memory is released
       if (ok && n_total > 0)
-        ok = mbar_wait(&bars[kDoFull], (n_total - 1) & 1, abort_flag, p.err, wait_tag(1, kDoFull, n_total - 1));
+        ok = mbar_wait(&bars[kDoFull], (n_total - 1) & 1, abort_flag, p.err, wait_tag(1, kDoFull, n_total - 1), p.wait_ns);
       if (!ok) drain_pause_ns(50000);   // let copies already issued land
     }
   } else if (warp == 9) {
@@ -257,23 +257,23 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         }
         umma_commit(&bars[kSFull]);
       };
-      bool ok = mbar_wait(&bars[kKVFull], 0, abort_flag, p.err, wait_tag(2, kKVFull, 0));
+      bool ok = mbar_wait(&bars[kKVFull], 0, abort_flag, p.err, wait_tag(2, kKVFull, 0), p.wait_ns);
       int n = 0, kc = 0, sk = 0;
       bool have_next = false;
-      if (ok) ok = mbar_wait(&bars[kQFull], 0, abort_flag, p.err, wait_tag(2, kQFull, 0));
+      if (ok) ok = mbar_wait(&bars[kQFull], 0, abort_flag, p.err, wait_tag(2, kQFull, 0), p.wait_ns);
       if (ok && misc[8] != kEndMarker) {
         tc_fence_after();
         issue_s(0);
         have_next = true;
       }
       while (ok && have_next) {
-        if (!mbar_wait(&bars[kDecFull], n & 1, abort_flag, p.err, wait_tag(2, kDecFull, n))) { ok = false; break; }
+        if (!mbar_wait(&bars[kDecFull], n & 1, abort_flag, p.err, wait_tag(2, kDecFull, n), p.wait_ns)) { ok = false; break; }
         const uint32_t keep = misc[5];
         mbar_arrive(&bars[kDecEmpty]);
         const int st = n & 1, stn = (n + 1) & 1;
         if (keep) {
-          if (!mbar_wait(&bars[kPtFull], kc & 1, abort_flag, p.err, wait_tag(2, kPtFull, kc))) { ok = false; break; }
-          if (!mbar_wait(&bars[kDoFull], n & 1, abort_flag, p.err, wait_tag(2, kDoFull, n))) { ok = false; break; }
+          if (!mbar_wait(&bars[kPtFull], kc & 1, abort_flag, p.err, wait_tag(2, kPtFull, kc), p.wait_ns)) { ok = false; break; }
+          if (!mbar_wait(&bars[kDoFull], n & 1, abort_flag, p.err, wait_tag(2, kDoFull, n), p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           // dV += P^T dO: A = P^T from TMEM (8 columns per 16 queries), B = dO MN-major
 #pragma unroll
@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
                          (kc > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&bars[kDvDone]);
           // dP^T = V_j dO^T into Y once the previous dQ part has left it
-          if (!mbar_wait(&bars[kYFree], (kc & 1) ^ 1, abort_flag, p.err, wait_tag(2, kYFree, kc))) { ok = false; break; }
+          if (!mbar_wait(&bars[kYFree], (kc & 1) ^ 1, abort_flag, p.err, wait_tag(2, kYFree, kc), p.wait_ns)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
@@ -292,15 +292,15 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
           umma_commit(&bars[kDpFull]);
           umma_commit(&bars[kDoEmpty]);
           // S^T of the next tile into X once dV has read P^T from it
-          if (!mbar_wait(&bars[kQFull + stn], ((n + 1) >> 1) & 1, abort_flag, p.err, wait_tag(2, kQFull + stn, n + 1))) { ok = false; break; }
+          if (!mbar_wait(&bars[kQFull + stn], ((n + 1) >> 1) & 1, abort_flag, p.err, wait_tag(2, kQFull + stn, n + 1), p.wait_ns)) { ok = false; break; }
           have_next = misc[8 + stn] != kEndMarker;
           if (have_next) {
-            if (!mbar_wait(&bars[kDvDone], kc & 1, abort_flag, p.err, wait_tag(2, kDvDone, kc))) { ok = false; break; }
+            if (!mbar_wait(&bars[kDvDone], kc & 1, abort_flag, p.err, wait_tag(2, kDvDone, kc), p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             issue_s(n + 1);
           }
           // dK += dS^T Q_i and the dQ part = dS K_j into Y
-          if (!mbar_wait(&bars[kDsFull], kc & 1, abort_flag, p.err, wait_tag(2, kDsFull, kc))) { ok = false; break; }
+          if (!mbar_wait(&bars[kDsFull], kc & 1, abort_flag, p.err, wait_tag(2, kDsFull, kc), p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t q = aQ + st * kTile;
 #pragma unroll
@@ -318,10 +318,10 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
           ++kc;
         } else {
           umma_commit(&bars[kQEmpty + st]);
-          if (!mbar_wait(&bars[kQFull + stn], ((n + 1) >> 1) & 1, abort_flag, p.err, wait_tag(2, kQFull + stn, n + 1))) { ok = false; break; }
+          if (!mbar_wait(&bars[kQFull + stn], ((n + 1) >> 1) & 1, abort_flag, p.err, wait_tag(2, kQFull + stn, n + 1), p.wait_ns)) { ok = false; break; }
           have_next = misc[8 + stn] != kEndMarker;
           if (have_next) {
-            if (!mbar_wait(&bars[kXRead], sk & 1, abort_flag, p.err, wait_tag(2, kXRead, sk))) { ok = false; break; }
+            if (!mbar_wait(&bars[kXRead], sk & 1, abort_flag, p.err, wait_tag(2, kXRead, sk), p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             issue_s(n + 1);
           }
@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
     // warp instruction cover 512 contiguous bytes; frees Y
     auto drain = [&]() {
       const bool okq = __all_sync(0xffffffffu, mbar_wait(&bars[kDqFull], (kc - 1) & 1, abort_flag, p.err,
-                                                          wait_tag(0, kDqFull, kc - 1)));
+                                                          wait_tag(0, kDqFull, kc - 1), p.wait_ns));
       uint32_t q0[32], q1[32];
       if (okq) {
         tc_fence_after();
@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
     while (true) {
       const int st = n & 1;
       const bool okq = __all_sync(0xffffffffu, mbar_wait(&bars[kQFull + st], (n >> 1) & 1, abort_flag, p.err,
-                                                         wait_tag(0, kQFull + st, n)));
+                                                         wait_tag(0, kQFull + st, n), p.wait_ns));
       const uint32_t qi = misc[8 + st];
       if (bar_or(1, 256, !okq || *abort_flag != 0) || qi == kEndMarker) break;
       const int i = static_cast<int>(qi);
@@ -403,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       // keeps them out of the test (-inf - t2 is -inf or NaN, and fmaxf
       // ignores NaN) and makes their P^T exactly 0. Padded query columns
       // carry t2 = z log2 e = +inf and drop out the same way.
-      const bool oks = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], n & 1, abort_flag, p.err, wait_tag(0, kSFull, n)));
+      const bool oks = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], n & 1, abort_flag, p.err, wait_tag(0, kSFull, n), p.wait_ns));
       uint32_t sr[2][32];
       if (oks) {
         tc_fence_after();
@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       const bool keep = bar_or(1, 256, vote);
       if (tid == 0) {
         misc[4] = (static_cast<uint32_t>(n) << 16) | (static_cast<uint32_t>(kc) & 0xffff);
-        if (mbar_wait(&bars[kDecEmpty], (n & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty, n))) {
+        if (mbar_wait(&bars[kDecEmpty], (n & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty, n), p.wait_ns)) {
           misc[5] = keep ? 1u : 0u;
           mbar_arrive(&bars[kDecFull]);
         }
@@ -493,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       if (pending) drain();
 
       // dS^T = P^T (dP^T - D) -> bf16 into this half's chunk of the dS^T tile
-      const bool okd = __all_sync(0xffffffffu, mbar_wait(&bars[kDpFull], kc & 1, abort_flag, p.err, wait_tag(0, kDpFull, kc)));
+      const bool okd = __all_sync(0xffffffffu, mbar_wait(&bars[kDpFull], kc & 1, abort_flag, p.err, wait_tag(0, kDpFull, kc), p.wait_ns));
       uint32_t dp[2][32];
       if (okd) {
         tc_fence_after();
@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
     if (pending && !*abort_flag) drain();
 
     // dK_j, dV_j (key row r, this half's 64 columns) -> bf16
-    const bool okdone = __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0, abort_flag, p.err, wait_tag(0, kDone, 0)));
+    const bool okdone = __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0, abort_flag, p.err, wait_tag(0, kDone, 0), p.wait_ns));
     const int krow = j * kB + r;
     if (okdone && !*abort_flag) {
       tc_fence_after();
@@ -584,6 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // after a timeout, copies issued before the waits gave up land before the
+  // CTA's shared memory is released
+  if (tid == 0 && *abort_flag) drain_pause_ns(50000);
 }
 
 // D = rowsum(dO o O), zl2 = z log2e, t2 = z + log tau - log(q + 1) (the

@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
       tma_prefetch_desc(&p.tm_k);
       for (int t = 0; t < T; ++t) {
         const int s = t % kNSK;
-        if (!mbar_wait(&bars[kKEmpty + s], ((t / kNSK) & 1) ^ 1, abort_flag, p.err, wait_tag(1, kKEmpty + s, t))) {
+        if (!mbar_wait(&bars[kKEmpty + s], ((t / kNSK) & 1) ^ 1, abort_flag, p.err, wait_tag(1, kKEmpty + s, t), p.wait_ns)) {
           drain_pause_ns(50000);         // copies already issued land before the CTA exits
           break;
         }
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
     auto do_pv = [&]() -> bool {
       const int s = pv_done % kNSV;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kVFull + s], (pv_done / kNSV) & 1, abort_flag,
-                                                         p.err, wait_tag(0, kVFull + s, pv_done)));
+                                                         p.err, wait_tag(0, kVFull + s, pv_done), p.wait_ns));
       if (ok) {
         const float pm_lo = sPendM[s * 16 + row_lo], pm_hi = sPendM[s * 16 + row_hi];
         const float f_lo = (pm_lo == om_lo) ? 1.0f : ex2_approx(om_lo - pm_lo);
@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
       const int j = t1 - 1 - t;
       const int ks = t % kNSK;
       const bool okk = __all_sync(0xffffffffu, mbar_wait(&bars[kKFull + ks], (t / kNSK) & 1, abort_flag, p.err,
-                                                         wait_tag(0, kKFull + ks, t)));
+                                                         wait_tag(0, kKFull + ks, t), p.wait_ns));
       float sacc[kNBW][4];
 #pragma unroll
       for (int nb = 0; nb < kNBW; ++nb)
@@ -434,7 +434,7 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
       if (kc - pv_done == kNSV) do_pv();
       const int s = kc % kNSV;
       const bool slot_ok = mbar_wait(&bars[kSlotFree + s], ((kc / kNSV) & 1) ^ 1, abort_flag, p.err,
-                                     wait_tag(0, kSlotFree + s, kc));
+                                     wait_tag(0, kSlotFree + s, kc), p.wait_ns);
       if (warp == 0 && lane == 0 && slot_ok) {
         // every warp has finished the slot's previous PV: load this tile's V
         mbar_expect_tx(&bars[kVFull + s], kRing);
@@ -529,6 +529,9 @@ __global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kern
     }
   }
   __syncthreads();
+  // after a timeout, copies issued before the waits gave up land before the
+  // CTA's shared memory is released
+  if (tid == 0 && *abort_flag) drain_pause_ns(50000);
 }
 
 // z = log sum_p exp(z_p), O = sum_p exp(z_p - z) O_p, one CTA per (b, head)

@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
           idle_since = global_timer_ns();
         } else if (*abort_flag) {
           ok = false;
-        } else if (global_timer_ns() - idle_since > kWaitLimitNs) {
+        } else if (global_timer_ns() - idle_since > p.wait_ns) {
           *abort_flag = 1;
           if (atomicCAS(p.err, 0, kErrTimeout) == 0) {
             p.err[1] = wait_tag(1, 0xff, next_d);
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       auto issue_qk = [&](int t) -> bool {
         const int ks = t % NK;
-        if (!mbar_wait(&bars[kKFull + ks], (t / NK) & 1, abort_flag, p.err, wait_tag(2, kKFull + ks, t))) return false;
+        if (!mbar_wait(&bars[kKFull + ks], (t / NK) & 1, abort_flag, p.err, wait_tag(2, kKFull + ks, t), p.wait_ns)) return false;
         tc_fence_after();
         const uint32_t sb = tmem + (t % kNS) * 128;
 #pragma unroll
@@ -295,18 +295,18 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
         misc[3] = 0x20000u | t;
         return true;
       };
-      bool ok = mbar_wait(&bars[kQFull], 0, abort_flag, p.err, wait_tag(2, kQFull, 0));
+      bool ok = mbar_wait(&bars[kQFull], 0, abort_flag, p.err, wait_tag(2, kQFull, 0), p.wait_ns);
       for (int t = 0; ok && t < kNS && t < T; ++t) ok = issue_qk(t);
       int kc = 0;
       for (int t = 0; ok && t < T; ++t) {
         const int ds = t & 1;
-        if (!mbar_wait(&bars[kDecFull + ds], (t >> 1) & 1, abort_flag, p.err, wait_tag(2, kDecFull + ds, t))) { ok = false; break; }
+        if (!mbar_wait(&bars[kDecFull + ds], (t >> 1) & 1, abort_flag, p.err, wait_tag(2, kDecFull + ds, t), p.wait_ns)) { ok = false; break; }
         const uint32_t keep = misc[5 + ds];
         mbar_arrive(&bars[kDecEmpty + ds]);
         if (keep) {
           const int vs = kc % NV;
-          if (!mbar_wait(&bars[kSDone + t % kNS], (t / kNS) & 1, abort_flag, p.err, wait_tag(2, kSDone + t % kNS, t))) { ok = false; break; }
-          if (!mbar_wait(&bars[kVFull + vs], (kc / NV) & 1, abort_flag, p.err, wait_tag(2, kVFull + vs, kc))) { ok = false; break; }
+          if (!mbar_wait(&bars[kSDone + t % kNS], (t / kNS) & 1, abort_flag, p.err, wait_tag(2, kSDone + t % kNS, t), p.wait_ns)) { ok = false; break; }
+          if (!mbar_wait(&bars[kVFull + vs], (kc / NV) & 1, abort_flag, p.err, wait_tag(2, kVFull + vs, kc), p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t pb = tmem + (t % kNS) * 128;   // P as packed bf16 pairs over S
 #pragma unroll
@@ -323,8 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
         // PV of a retained tile) has completed
         if (t + kNS < T) {
           if (!keep &&
-              !mbar_wait(&bars[kSDone + t % kNS], (t / kNS) & 1, abort_flag, p.err, wait_tag(2, kSDone + t % kNS, t))) { ok = false; break; }
-          if (!mbar_wait(&bars[kTileDone + t % kNS], (t / kNS) & 1, abort_flag, p.err, wait_tag(2, kTileDone + t % kNS, t))) { ok = false; break; }
+              !mbar_wait(&bars[kSDone + t % kNS], (t / kNS) & 1, abort_flag, p.err, wait_tag(2, kSDone + t % kNS, t), p.wait_ns)) { ok = false; break; }
+          if (!mbar_wait(&bars[kTileDone + t % kNS], (t / kNS) & 1, abort_flag, p.err, wait_tag(2, kTileDone + t % kNS, t), p.wait_ns)) { ok = false; break; }
           if (!issue_qk(t + kNS)) { ok = false; break; }
         }
       }
@@ -363,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       uint32_t sr[2][32];
       // tcgen05.ld is warp-collective: load only if every lane's wait succeeded
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull + sb], (t / kNS) & 1, abort_flag, p.err,
-                                                        wait_tag(0, kSFull + sb, t)));
+                                                        wait_tag(0, kSFull + sb, t), p.wait_ns));
       if (ok) {
         tc_fence_after();
         tmem_ld32(tmem + sb * 128 + lane_addr + c0, sr[0]);
@@ -416,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
         // wait moves to the next tile's exchange, off the critical path.
         if (pending >= 0) {
           mbar_wait<true>(&cbars[pending & 1], (pending >> 1) & 1, abort_flag, p.err,
-                          wait_tag(0, 0x40 + (pending & 1), pending));
+                          wait_tag(0, 0x40 + (pending & 1), pending), p.wait_ns);
           pending = -1;
         }
         if (tid < p.group) {          // one lane per peer, in parallel
@@ -426,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
         }
         if (keep) {
           pending = t;
-        } else if (mbar_wait<true>(&cbars[par], (t >> 1) & 1, abort_flag, p.err, wait_tag(0, 0x40 + par, t))) {
+        } else if (mbar_wait<true>(&cbars[par], (t >> 1) & 1, abort_flag, p.err, wait_tag(0, 0x40 + par, t), p.wait_ns)) {
           bool any = false;
           for (int rr = 0; rr < p.group; ++rr) any = any || cvote[par * 8 + rr] != 0u;
           keep = any;
@@ -434,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       }
 
       if (tid == 0) {
-        if (mbar_wait(&bars[kDecEmpty + par], ((t >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty + par, t))) {
+        if (mbar_wait(&bars[kDecEmpty + par], ((t >> 1) & 1) ^ 1, abort_flag, p.err, wait_tag(0, kDecEmpty + par, t), p.wait_ns)) {
           misc[5 + par] = keep ? 1u : 0u;
           mbar_arrive(&bars[kDecFull + par]);
         }
@@ -473,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
         // O holds the PVs of earlier retained tiles: wait until every MMA up
         // to the previous tile has completed (t >= 1 since kc > 0)
         const int tp = t - 1;
-        mbar_wait(&bars[kTileDone + tp % kNS], (tp / kNS) & 1, abort_flag, p.err, wait_tag(0, kTileDone + tp % kNS, tp));
+        mbar_wait(&bars[kTileDone + tp % kNS], (tp / kNS) & 1, abort_flag, p.err, wait_tag(0, kTileDone + tp % kNS, tp), p.wait_ns);
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
@@ -521,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       if (prev_kept) l += xsum[(((T - 1) & 1) * 2 + 0) * 128 + r] + xsum[(((T - 1) & 1) * 2 + 1) * 128 + r];
       if (kc > 0)
         mbar_wait(&bars[kTileDone + (T - 1) % kNS], ((T - 1) / kNS) & 1, abort_flag, p.err,
-                  wait_tag(0, kTileDone + (T - 1) % kNS, T - 1));
+                  wait_tag(0, kTileDone + (T - 1) % kNS, T - 1), p.wait_ns);
       tc_fence_after();
       const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + static_cast<int64_t>(tb) * p.o_sb +
@@ -566,6 +566,9 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // after a timeout, copies issued before the waits gave up land before the
+  // CTA's shared memory is released
+  if (tid == 0 && *abort_flag) drain_pause_ns(50000);
   // no CTA leaves while a peer may still write to its shared memory
   if (p.group_vote) cluster_sync_all();
 }

@@ -43,6 +43,7 @@ struct FwdTcParams {
   int group;            // G = Hq / Hkv
   int group_vote;       // group-joint voting: the G CTAs of a query block's
                         // KV-head group form one cluster (G <= 8)
+  uint64_t wait_ns;     // limit of every bounded wait (ns)
 };
 
 cudaError_t launch_fwd_tc(const FwdTcParams& p, int head_dim, cudaStream_t stream);
@@ -92,6 +93,7 @@ struct DecodeParams {
   int group_vote;       // one decision per key tile for the whole query-head group
   uint8_t group_size[kMaxKvHeads];
   uint8_t group_heads[kMaxKvHeads][kMaxGroup];
+  uint64_t wait_ns;     // limit of every bounded wait (ns)
 };
 
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
@@ -115,6 +117,7 @@ struct BwdParams {
   uint8_t group_size[kMaxKvHeads];
   uint8_t group_heads[kMaxKvHeads][kMaxGroup];
   SeqTable seq;            // packed sequences (B = their number; nQB / nKB maxima)
+  uint64_t wait_ns;        // limit of every bounded wait (ns)
 };
 
 struct BwdAuxParams {      // pre-pass and dQ conversion

@@ -111,6 +111,13 @@ int* device_error_ptr() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Wait limit of a call's kernels: the caller's value, or 2 s for 0.
+int wait_limit(int64_t ns, uint64_t* out) {
+  if (ns < 0) return fail(MALA_ERR_INVALID_ARG, "wait_limit_ns %lld is negative", (long long)ns);
+  *out = ns == 0 ? 2000000000ull : static_cast<uint64_t>(ns);
+  return MALA_OK;
+}
+
 // Checks one [B, N, H, d] operand: non-NULL, 16-byte aligned, strides
 // non-negative multiples of 16 bytes, rows that do not overlap.
 int check_tensor(const char* name, const void* p, const int64_t* st, int64_t esize, int64_t d,
@@ -232,6 +239,7 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
   if (!a) return fail(MALA_ERR_INVALID_ARG, "args is NULL");
   int rc = check_common(a->batch, a->heads_q, a->heads_kv, a->head_dim, a->tau, a->dtype);
   if (rc) return rc;
+  if (a->wait_limit_ns < 0) return fail(MALA_ERR_INVALID_ARG, "wait_limit_ns %lld is negative", (long long)a->wait_limit_ns);
   if (a->mode != MALA_CAUSAL)
     return fail(MALA_ERR_UNSUPPORTED, "mala_fwd supports MALA_CAUSAL; use mala_decode for decoding");
   if (a->seqlen_q <= 0 || a->seqlen_k <= 0) return fail(MALA_ERR_INVALID_ARG, "sequence lengths must be positive");
@@ -298,6 +306,7 @@ int mala_fwd(const mala_fwd_args* a, void* workspace, size_t ws_bytes, void* str
     if ((rc = make_map_bf16(&p.tm_k, a->k, mb, Nk, a->heads_kv, d, a->k_stride, 128))) return rc;
     if ((rc = make_map_bf16(&p.tm_v, a->v, mb, Nk, a->heads_kv, d, a->v_stride, 128))) return rc;
     p.seq = seq;
+    if ((rc = wait_limit(a->wait_limit_ns, &p.wait_ns))) return rc;
     p.err = device_error_ptr();
     if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
     p.o = a->o;
@@ -359,6 +368,7 @@ namespace {
 int bwd_check(const mala_bwd_args* a) {
   int rc = check_common(a->batch, a->heads_q, a->heads_kv, a->head_dim, a->tau, a->dtype);
   if (rc) return rc;
+  if (a->wait_limit_ns < 0) return fail(MALA_ERR_INVALID_ARG, "wait_limit_ns %lld is negative", (long long)a->wait_limit_ns);
   if (a->dtype != MALA_BF16) return fail(MALA_ERR_UNSUPPORTED, "backward supports bf16 only");
   if (a->head_dim != 128) return fail(MALA_ERR_UNSUPPORTED, "backward supports head_dim 128 only");
   if (a->block_q != 128 || a->block_k != 128) return fail(MALA_ERR_UNSUPPORTED, "backward supports 128 x 128 tiles only");
@@ -452,6 +462,7 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
   p.fwd_mask = a->keep_mask;
   p.bwd_mask = a->bwd_keep_mask;
   p.stats = a->stats;
+  if ((rc = wait_limit(a->wait_limit_ns, &p.wait_ns))) return rc;
   p.err = device_error_ptr();
   if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
   p.dk_sb = a->dk_stride[0]; p.dk_sn = a->dk_stride[1]; p.dk_sh = a->dk_stride[2];
@@ -515,6 +526,7 @@ int decode_check(const mala_decode_args* a, int* nKB_out) {
   if (a->seqlen_k > (1 << 30)) return fail(MALA_ERR_UNSUPPORTED, "cache too long");
   if (a->heads_kv > mala::kMaxKvHeads) return fail(MALA_ERR_UNSUPPORTED, "heads_kv > %d", mala::kMaxKvHeads);
   if (!a->lse) return fail(MALA_ERR_INVALID_ARG, "lse is NULL");
+  if (a->wait_limit_ns < 0) return fail(MALA_ERR_INVALID_ARG, "wait_limit_ns %lld is negative", (long long)a->wait_limit_ns);
   const int nKB = static_cast<int>((a->seqlen_k + 127) / 128);
   if (a->num_splits < 0 || a->num_splits > nKB)
     return fail(MALA_ERR_INVALID_ARG, "num_splits %d outside [0, %d]", a->num_splits, nKB);
@@ -591,6 +603,7 @@ int decode_launch(mala_decode_args* a, int nKB, int P, float* partials, void* st
   }
   if ((rc = decode_cache_maps(a, &p))) return rc;
   p.group_vote = a->group_vote;
+  if ((rc = wait_limit(a->wait_limit_ns, &p.wait_ns))) return rc;
   p.err = device_error_ptr();
   if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
   p.q = a->q;

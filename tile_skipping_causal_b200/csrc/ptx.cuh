@@ -92,6 +92,32 @@ __device__ __forceinline__ bool mbar_test_cluster(uint64_t* bar, uint32_t parity
   return ok != 0;
 }
 
+// try_wait whose suspension lasts at most hint_ns (instead of the hardware's
+// own limit), so that a short wait limit is checked within that time
+__device__ __forceinline__ bool mbar_test_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_test_cluster_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // ---- thread-block clusters (distributed shared memory)
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -122,23 +148,37 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 
 // Wait for the phase of `bar` with parity `parity` to complete. Gives up
-// when *abort becomes non-zero (another thread gave up) or after
-// kWaitLimitNs; then sets *abort and records the timeout in the error block
+// when *abort becomes non-zero (another thread gave up) or after limit_ns
+// nanoseconds (the call's wait limit, kWaitLimitNs unless the caller set
+// one); then sets *abort and records the timeout in the error block
 // err[0..6] = {code, tag of the first wait that gave up, its block index,
 // its parity, progress words abort[1..3]}. `tag` identifies the wait site
 // (role, barrier, tile); abort[1..3] must be readable shared words.
 // kCluster: acquire at cluster scope (for arrivals from other CTAs).
+// A limit below kWaitLimitNs (set by a caller that tests this path) also
+// bounds each try_wait's own suspension, so that even a wait the hardware
+// would satisfy within one suspension is measured against the limit.
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort, int* err, int tag = 0) {
-  auto test = [&]() { return kCluster ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity); };
+                                          volatile int* abort, int* err, int tag,
+                                          uint64_t limit_ns) {
+  const bool short_limit = limit_ns < kWaitLimitNs;
+  const uint32_t hint = static_cast<uint32_t>(limit_ns < 1000000ull ? limit_ns : 1000000ull);
+  auto test = [&]() {
+    if (short_limit)
+      return kCluster ? mbar_test_cluster_hint(bar, parity, hint) : mbar_test_hint(bar, parity, hint);
+    return kCluster ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity);
+  };
   if (test()) return true;
   uint64_t t0 = global_timer_ns();
+  // the abort flag and the clock are read every 64 tries, every try under a
+  // short limit
+  const uint32_t check_mask = short_limit ? 0u : 63u;
   for (uint32_t it = 1;; ++it) {
     if (test()) return true;
-    if ((it & 63u) == 0) {
+    if ((it & check_mask) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort = 1;
         if (atomicCAS(err, 0, kErrTimeout) == 0) {
           err[1] = tag;

@@ -36,7 +36,7 @@ class FwdArgs(ctypes.Structure):
         ("q_to_kv", ctypes.c_void_p), ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32),
         ("tau", ctypes.c_float), ("dtype", ctypes.c_int32), ("mode", ctypes.c_int32),
         ("stats", ctypes.c_void_p), ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
-        ("group_vote", ctypes.c_int32),
+        ("group_vote", ctypes.c_int32), ("wait_limit_ns", ctypes.c_int64),
     ]
 
 
@@ -53,6 +53,7 @@ class BwdArgs(ctypes.Structure):
         ("q_to_kv", ctypes.c_void_p), ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32),
         ("tau", ctypes.c_float), ("dtype", ctypes.c_int32), ("stats", ctypes.c_void_p),
         ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+        ("wait_limit_ns", ctypes.c_int64),
     ]
 
 
@@ -66,7 +67,7 @@ class DecodeArgs(ctypes.Structure):
         ("q_to_kv", ctypes.c_void_p), ("block_k", ctypes.c_int32), ("tau", ctypes.c_float),
         ("dtype", ctypes.c_int32), ("num_splits", ctypes.c_int32), ("stats", ctypes.c_void_p),
         ("kv_dtype", ctypes.c_int32), ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
-        ("group_vote", ctypes.c_int32),
+        ("group_vote", ctypes.c_int32), ("wait_limit_ns", ctypes.c_int64),
     ]
 
 
@@ -236,7 +237,7 @@ def _packed(cu_seqlens_q, cu_seqlens_k, block_q, block_k):
 def mala_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float,
              block_q: int = 128, block_k: int = 128, *, o=None, lse=None, keep_mask=None,
              with_mask: bool = True, stats=None, q_to_kv=None, stream=None,
-             cu_seqlens_q=None, cu_seqlens_k=None, group_vote: bool = False):
+             cu_seqlens_q=None, cu_seqlens_k=None, group_vote: bool = False, wait_limit_ns: int = 0):
     """MALA forward/prefill. q [B, N_q, Hq, d], k/v [B, N_k, Hkv, d] (bf16 or
     fp32, scale folded into q; N_q <= N_k, bottom-right aligned). Returns
     (o, lse [B, Hq, N_q] fp32, keep_mask words [B, Hq, nQB, ceil(nKB/32)]
@@ -250,7 +251,10 @@ def mala_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float,
     group_vote: one decision per (query block, key tile) for the query heads
     of a KV head (a tile is skipped only when every row of every head passes
     the test; bf16, 128 x 128 tiles, default head map, at most 8 heads per
-    group)."""
+    group).
+
+    wait_limit_ns: limit of every device-side wait (0 = the library's 2 s);
+    small values only serve tests of the timeout path."""
     lib = load_library()
     _require_cuda(q, k, v)
     B, N, Hq, d = q.shape
@@ -271,6 +275,7 @@ def mala_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float,
     keep_alive, hm = _head_map(q_to_kv)
     a = fwd_args(q, k, v, o, lse, keep_mask, tau, block_q, block_k, stats, hm)
     a.group_vote = 1 if group_vote else 0
+    a.wait_limit_ns = int(wait_limit_ns)
     if packed:
         a.batch = packed[2]
         a.cu_seqlens_q = packed[0].ctypes.data
@@ -286,10 +291,10 @@ def mala_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tau: float,
 def mala_bwd(q, k, v, o, do, lse, tau: float, keep_mask=None, block_q: int = 128,
              block_k: int = 128, *, dq=None, dk=None, dv=None, bwd_keep_mask=None,
              with_bwd_mask: bool = False, stats=None, q_to_kv=None, stream=None,
-             cu_seqlens_q=None, cu_seqlens_k=None):
+             cu_seqlens_q=None, cu_seqlens_k=None, wait_limit_ns: int = 0):
     """MALA backward. Returns (dq, dk, dv, bwd_keep_mask or None). Packed
     sequences as for mala_fwd (the same cu_seqlens; lse and keep_mask in
-    mala_fwd's packed layouts)."""
+    mala_fwd's packed layouts). wait_limit_ns as for mala_fwd."""
     lib = load_library()
     _require_cuda(q, k, v, o, do, lse)
     B, N, Hq, d = q.shape
@@ -320,6 +325,7 @@ def mala_bwd(q, k, v, o, do, lse, tau: float, keep_mask=None, block_q: int = 128
     a.tau = float(tau)
     a.dtype = _dtype_code(q)
     a.stats = _ptr(stats)
+    a.wait_limit_ns = int(wait_limit_ns)
     if packed:
         a.batch = packed[2]
         a.cu_seqlens_q = packed[0].ctypes.data
@@ -344,7 +350,7 @@ def _decode_cache(a, k, v, k_scale, v_scale):
 
 
 def _decode_call(q, k, v, tau, block_k, num_splits, o, lse, keep_mask, with_mask, stats, q_to_kv,
-                 k_scale, v_scale, group_vote):
+                 k_scale, v_scale, group_vote, wait_limit_ns=0):
     """Output tensors and the filled argument struct of a decode call (plus
     the objects that must outlive the call)."""
     _require_cuda(q, k, v)
@@ -369,22 +375,24 @@ def _decode_call(q, k, v, tau, block_k, num_splits, o, lse, keep_mask, with_mask
     a.stats = _ptr(stats)
     _decode_cache(a, k, v, k_scale, v_scale)
     a.group_vote = 1 if group_vote else 0
+    a.wait_limit_ns = int(wait_limit_ns)
     return o, lse, keep_mask, a, keep_alive
 
 
 def mala_decode(q, k, v, tau: float, block_k: int = 128, num_splits: int = 0, *, o=None,
                 lse=None, keep_mask=None, with_mask: bool = True, stats=None, q_to_kv=None,
                 stream=None, workspace=None, k_scale: float = 1.0, v_scale: float = 1.0,
-                group_vote: bool = False):
+                group_vote: bool = False, wait_limit_ns: int = 0):
     """Single-token decoding. q [B, 1, Hq, d] bf16; k/v cache [B, Nk, Hkv, d]
     in bf16, or torch.float8_e4m3fn codes whose values are code * k_scale and
     code * v_scale. group_vote: one decision per key tile for all query heads
     of a KV head (a tile is skipped only when every head passes the test).
-    Returns (o, lse [B, Hq], keep_mask words [B, Hq, ceil(T/32)] or None,
-    num_splits used)."""
+    wait_limit_ns as for mala_fwd. Returns (o, lse [B, Hq], keep_mask words
+    [B, Hq, ceil(T/32)] or None, num_splits used)."""
     lib = load_library()
     o, lse, keep_mask, a, keep_alive = _decode_call(q, k, v, tau, block_k, num_splits, o, lse, keep_mask,
-                                                    with_mask, stats, q_to_kv, k_scale, v_scale, group_vote)
+                                                    with_mask, stats, q_to_kv, k_scale, v_scale, group_vote,
+                                                    wait_limit_ns)
     ws_n = lib.mala_decode_workspace_size(ctypes.byref(a))
     own_ws = workspace is None or workspace.numel() < ws_n
     if own_ws:
