@@ -414,9 +414,14 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
         // peer rewrites a vote slot before this CTA has read it. When this
         // CTA's own vote already retains the tile, the OR is known and the
         // wait moves to the next tile's exchange, off the critical path.
+        // The deferred wait only orders this CTA's sends, so only warp 0
+        // (whose lanes send) takes it; every thread that reads the vote
+        // slots of a tile has done so before the next tile's vote barrier,
+        // which precedes the next send.
         if (pending >= 0) {
-          mbar_wait<true>(&cbars[pending & 1], (pending >> 1) & 1, abort_flag, p.err,
-                          wait_tag(0, 0x40 + (pending & 1), pending), p.wait_ns);
+          if (warp == 0)
+            mbar_wait<true>(&cbars[pending & 1], (pending >> 1) & 1, abort_flag, p.err,
+                            wait_tag(0, 0x40 + (pending & 1), pending), p.wait_ns);
           pending = -1;
         }
         if (tid < p.group) {          // one lane per peer, in parallel
