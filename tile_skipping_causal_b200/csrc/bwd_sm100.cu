@@ -54,11 +54,14 @@ struct Smem {
   static constexpr uint32_t kQ = kV + kTile;                // 2 stages
   static constexpr uint32_t kDO = kQ + 2 * kTile;
   static constexpr uint32_t kDS = kDO + kTile;
-  static constexpr uint32_t kStats = kDS + kTile;           // [2 stages][zl2, t2, D][128]
-  static constexpr uint32_t kBars = kStats + 2 * 3 * 128 * 4;
+  static constexpr uint32_t kStage = kDS + kTile;           // dQ staging: 16 KB per compute warpgroup
+  static constexpr uint32_t kStats = kStage + kTile;        // [2 stages][zl2, D][128]
+  static constexpr uint32_t kBars = kStats + 2 * 2 * 128 * 4;
   static constexpr uint32_t kMisc = kBars + kNumBars * 8;
   static constexpr uint32_t kEnd = kMisc + 64;
-  static constexpr uint32_t kAlloc = kEnd + 1024;
+  // the dynamic shared memory base is 1024-byte aligned (checked at entry),
+  // as the 128-byte swizzled TMA tiles require
+  static constexpr uint32_t kAlloc = kEnd;
 };
 static_assert(Smem::kAlloc > 116 * 1024, "backward CTA must exclude a second resident CTA per SM");
 static_assert(Smem::kAlloc <= 232448, "backward CTA exceeds shared memory");
@@ -69,14 +72,19 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_constant__ BwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    // every thread sees the same address: a uniform exit before any barrier
+    if (threadIdx.x == 0) atomicCAS(p.err, 0, kErrSmemAlign);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sK = smem + Smem::kK;
   uint8_t* sV = smem + Smem::kV;
   uint8_t* sQ = smem + Smem::kQ;
   uint8_t* sDO = smem + Smem::kDO;
   uint8_t* sDS = smem + Smem::kDS;
+  uint8_t* sStage = smem + Smem::kStage;
   float* sStats = reinterpret_cast<float*>(smem + Smem::kStats);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::kBars);
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + Smem::kMisc);
@@ -181,14 +189,13 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         info_i[n & 3] = i;
         misc[6 + st] = static_cast<uint32_t>(h);
         misc[8 + st] = static_cast<uint32_t>(i);
-        mbar_expect_tx(&bars[kQFull + st], kTile + 3 * 512);
+        mbar_expect_tx(&bars[kQFull + st], kTile + 2 * 512);
         for (int c = 0; c < 2; ++c)
           tma_load_4d(sQ + st * kTile + c * kChunk, &p.tm_q, &bars[kQFull + st], c * 64, h, qrow0 + i * kB, tb);
         const int64_t row0 = qblock_index(p.seq, p.Hq, p.nQB, b, h, i) * kB;
-        float* sst = sStats + st * 384;
+        float* sst = sStats + st * 256;
         bulk_load(sst, p.zl2 + row0, 512, &bars[kQFull + st]);
-        bulk_load(sst + 128, p.t2 + row0, 512, &bars[kQFull + st]);
-        bulk_load(sst + 256, p.Dv + row0, 512, &bars[kQFull + st]);
+        bulk_load(sst + 128, p.Dv + row0, 512, &bars[kQFull + st]);
         return true;
       };
       // In order, with blocking waits. dO of tile n + 1 is loaded one tile
@@ -352,9 +359,14 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
     int pend_h = 0, pend_i = 0;
 
     // dQ part of the previous retained tile (query row r, this half's 64
-    // columns): TMEM -> registers -> vector fp32 reductions into the
-    // accumulator, whose layout [.., 32 column quads, 128 rows, 4] makes each
-    // warp instruction cover 512 contiguous bytes; frees Y
+    // columns): TMEM -> registers (Y is then free) -> this warpgroup's 16 KB
+    // staging buffer in the accumulator's blocked layout [.., 32 column
+    // quads, 128 rows, 4] -> one asynchronous bulk fp32 reduction per 32
+    // columns (16 KB contiguous in the accumulator), issued by one thread of
+    // the warpgroup, in place of one vector reduction per thread and 16
+    // bytes. Before a warpgroup refills its buffer, its leader waits until
+    // the previous bulk reduction has read it.
+    const bool wg_leader = (warp & 3) == 0 && lane == 0;
     auto drain = [&]() {
       const bool okq = __all_sync(0xffffffffu, mbar_wait(&bars[kDqFull], (kc - 1) & 1, abort_flag, p.err,
                                                           wait_tag(0, kDqFull, kc - 1), p.wait_ns));
@@ -372,15 +384,25 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       reg_fence(q1);
       tc_fence_before();
       warp_arrive(&bars[kYFree]);
-      float* dst = p.dq_acc + qblock_index(p.seq, p.Hq, p.nQB, b, pend_h, pend_i) * (kB * kD) + r * 4;
+      float* dst = p.dq_acc + qblock_index(p.seq, p.Hq, p.nQB, b, pend_h, pend_i) * (kB * kD);
+      uint8_t* stg = sStage + half * 16384;
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        red_add_v4_f32(dst + (c0 / 4 + u) * (kB * 4), __uint_as_float(q0[4 * u]), __uint_as_float(q0[4 * u + 1]),
-                       __uint_as_float(q0[4 * u + 2]), __uint_as_float(q0[4 * u + 3]));
+      for (int c = 0; c < 2; ++c) {
+        const uint32_t* q = c ? q1 : q0;
+        // the previous reduction from this half has finished reading it
+        if (wg_leader) bulk_wait_read<0>();
+        named_bar_sync(2 + half, 128);
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        red_add_v4_f32(dst + (c0 / 4 + 8 + u) * (kB * 4), __uint_as_float(q1[4 * u]), __uint_as_float(q1[4 * u + 1]),
-                       __uint_as_float(q1[4 * u + 2]), __uint_as_float(q1[4 * u + 3]));
+        for (int u = 0; u < 8; ++u)
+          st_shared_v4(smem_u32(stg) + (u * kB + r) * 16, q[4 * u], q[4 * u + 1], q[4 * u + 2], q[4 * u + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(2 + half, 128);
+        if (wg_leader) {
+          // quads [16 half + 8c, + 8): 32 columns, 16 KB contiguous
+          bulk_reduce_add_f32(dst + (16 * half + 8 * c) * (kB * 4), stg, 16384);
+          bulk_commit_group();
+        }
+      }
       pending = false;
     };
 
@@ -392,17 +414,16 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       if (bar_or(1, 256, !okq || *abort_flag != 0) || qi == kEndMarker) break;
       const int i = static_cast<int>(qi);
       const int h = static_cast<int>(misc[6 + st]);
-      const float4* zl2_4 = reinterpret_cast<const float4*>(sStats + st * 384 + c0);
-      const float4* thr_4 = reinterpret_cast<const float4*>(sStats + st * 384 + 128 + c0);
-      const float4* dv_4 = reinterpret_cast<const float4*>(sStats + st * 384 + 256 + c0);
-      // test over this half of the S^T row: retain iff some legal entry has
-      // s - t2 >= 0 (t2 = z + log tau - log L_q of the entry's query
-      // column). Illegal entries (keys after the query's position, and key
-      // rows past N_k) only occur in tiles whose last key lies beyond the
+      const float4* zl2_4 = reinterpret_cast<const float4*>(sStats + st * 256 + c0);
+      const float4* dv_4 = reinterpret_cast<const float4*>(sStats + st * 256 + 128 + c0);
+      // test over this half of the S^T row, in log2 units: retain iff some
+      // legal entry has u + log2 L_q >= log2 tau, with u = s log2 e - z log2 e
+      // (also the exponent of P^T) and L_q = position + 1 of the entry's
+      // query column. Illegal entries (keys after the query's position, and
+      // key rows past N_k) only occur in tiles whose last key lies beyond the
       // block's first query position; there they are set to -inf once, which
-      // keeps them out of the test (-inf - t2 is -inf or NaN, and fmaxf
-      // ignores NaN) and makes their P^T exactly 0. Padded query columns
-      // carry t2 = z log2 e = +inf and drop out the same way.
+      // makes u = -inf: they drop out of the test and their P^T is exactly 0.
+      // Padded query columns carry z log2 e = +inf and drop out the same way.
       const bool oks = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], n & 1, abort_flag, p.err, wait_tag(0, kSFull, n), p.wait_ns));
       uint32_t sr[2][32];
       if (oks) {
@@ -424,22 +445,41 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
         for (int x = 0; x < 64; ++x)
           if (x < lim) sr[x >> 5][x & 31] = __float_as_uint(-INFINITY);
       }
-      float mx[8];
+      // u kept in sr as the exponent of P^T. L_q of this half's columns lies
+      // in [L0, L0 + 63], so with M = max u the row retains when
+      // M + log2 L0 >= log2 tau and skips when M + log2(L0 + 63) < log2 tau;
+      // only between the two bounds is each entry tested on its own. A row
+      // without a legal entry (M = -inf) never retains.
+      float mu[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+      for (int e = 0; e < 8; ++e) mu[e] = -INFINITY;
 #pragma unroll
       for (int x4 = 0; x4 < 16; ++x4) {
-        const float4 tv = thr_4[x4];
-        const float th[4] = {tv.x, tv.y, tv.z, tv.w};
+        const float4 zv = zl2_4[x4];
+        const float zz[4] = {zv.x, zv.y, zv.z, zv.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int x = 4 * x4 + e;
-          mx[x & 7] = fmaxf(mx[x & 7], __uint_as_float(sr[x >> 5][x & 31]) - th[e]);
+          const float u = fmaf(__uint_as_float(sr[x >> 5][x & 31]), kLog2e, -zz[e]);
+          sr[x >> 5][x & 31] = __float_as_uint(u);
+          mu[x & 7] = fmaxf(mu[x & 7], u);
         }
       }
-      const float mall = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      const bool vote = mall >= 0.0f;
+      const float M = fmaxf(fmaxf(fmaxf(mu[0], mu[1]), fmaxf(mu[2], mu[3])),
+                            fmaxf(fmaxf(mu[4], mu[5]), fmaxf(mu[6], mu[7])));
+      const float L0 = static_cast<float>(i * kB + c0 + q_off + 1);   // L_q of column c0
+      bool vote;
+      if (!(M > -INFINITY) || M + lg2_approx(L0 + 63.0f) < p.log2_tau) {
+        vote = false;
+      } else if (M + lg2_approx(L0) >= p.log2_tau) {
+        vote = true;
+      } else {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < 64; ++x)
+          mx = fmaxf(mx, __uint_as_float(sr[x >> 5][x & 31]) + lg2_approx(L0 + static_cast<float>(x)));
+        vote = mx >= p.log2_tau;
+      }
       const bool keep = bar_or(1, 256, vote);
       if (tid == 0) {
         misc[4] = (static_cast<uint32_t>(n) << 16) | (static_cast<uint32_t>(kc) & 0xffff);
@@ -472,18 +512,9 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       // columns [32 half, 32 half + 32) may overwrite either half's S^T.
       uint32_t pp[32];
 #pragma unroll
-      for (int x4 = 0; x4 < 16; ++x4) {
-        const float4 zv = zl2_4[x4];
-        const float zz[4] = {zv.x, zv.y, zv.z, zv.w};
-        float pv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int x = 4 * x4 + e;
-          pv[e] = ex2_approx(fmaf(__uint_as_float(sr[x >> 5][x & 31]), kLog2e, -zz[e]));
-        }
-        pp[2 * x4] = pack_bf16x2(pv[0], pv[1]);
-        pp[2 * x4 + 1] = pack_bf16x2(pv[2], pv[3]);
-      }
+      for (int x2 = 0; x2 < 32; ++x2)
+        pp[x2] = pack_bf16x2(ex2_approx(__uint_as_float(sr[(2 * x2) >> 5][(2 * x2) & 31])),
+                             ex2_approx(__uint_as_float(sr[(2 * x2 + 1) >> 5][(2 * x2 + 1) & 31])));
       tmem_st16(tX + lane_addr + half * 32, &pp[0]);
       tmem_st16(tX + lane_addr + half * 32 + 16, &pp[16]);
       tmem_st_wait();
@@ -537,7 +568,12 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       ++kc;
       ++n;
     }
-    if (pending && !*abort_flag) drain();
+    // the drain synchronises each warpgroup on a named barrier, so every
+    // compute thread must take the same branch: decide by a vote
+    if (!bar_or(1, 256, *abort_flag != 0) && pending) drain();
+    // the bulk reductions into the dQ accumulator complete before the CTA
+    // exits (the conversion kernel reads the accumulator next)
+    if (wg_leader) bulk_wait_all<0>();
 
     // dK_j, dV_j (key row r, this half's 64 columns) -> bf16
     const bool okdone = __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0, abort_flag, p.err, wait_tag(0, kDone, 0), p.wait_ns));
@@ -589,13 +625,12 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
   if (tid == 0 && *abort_flag) drain_pause_ns(50000);
 }
 
-// D = rowsum(dO o O), zl2 = z log2e, t2 = z + log tau - log(q + 1) (the
-// score a legal entry must reach to retain the tile, natural log units),
-// padded rows: zl2 = t2 = +inf, D = 0; zero the block's dQ accumulator.
+// D = rowsum(dO o O), zl2 = z log2e; padded rows: zl2 = +inf, D = 0; zero
+// the block's dQ accumulator.
 // Query block of an auxiliary CTA: blk = qblock_index(b, h, i); the
-// sequence's first query row, batch coordinate, length and offset.
+// sequence's first query row, batch coordinate and length.
 struct AuxBlock {
-  int b, h, i, qrow0, tb, Nq, q_off;
+  int b, h, i, qrow0, tb, Nq;
 };
 
 __device__ __forceinline__ AuxBlock aux_block(const BwdAuxParams& p, int blk) {
@@ -608,7 +643,6 @@ __device__ __forceinline__ AuxBlock aux_block(const BwdAuxParams& p, int blk) {
     a.qrow0 = 0;
     a.tb = a.b;
     a.Nq = p.N;
-    a.q_off = p.q_off;
   } else {
     const int QB = p.seq.qb0[p.seq.n];
     a.h = blk / QB;
@@ -624,7 +658,6 @@ __device__ __forceinline__ AuxBlock aux_block(const BwdAuxParams& p, int blk) {
     a.qrow0 = p.seq.q0[lo];
     a.tb = 0;
     a.Nq = p.seq.q0[lo + 1] - a.qrow0;
-    a.q_off = (p.seq.k0[lo + 1] - p.seq.k0[lo]) - a.Nq;
   }
   return a;
 }
@@ -661,11 +694,9 @@ __global__ void __launch_bounds__(128) mala_bwd_pre_kernel(const __grid_constant
                                  : p.lse[static_cast<int64_t>(h) * p.seq.q0[p.seq.n] + qr];
     p.Dv[row] = acc;
     p.zl2[row] = z * kLog2e;
-    p.t2[row] = z + p.log_tau - logf(static_cast<float>(q + ab.q_off + 1));
   } else {
     p.Dv[row] = 0.0f;
     p.zl2[row] = INFINITY;
-    p.t2[row] = INFINITY;
   }
   float4* acc4 = reinterpret_cast<float4*>(p.dq_acc + static_cast<int64_t>(blk) * (kB * kD));
   for (int e = t; e < kB * kD / 4; e += 128) acc4[e] = make_float4(0.f, 0.f, 0.f, 0.f);

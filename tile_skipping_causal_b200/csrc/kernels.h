@@ -10,6 +10,11 @@ namespace mala {
 
 constexpr int kMaxHeads = 256;
 
+// Code a kernel writes to the library's device error word when its dynamic
+// shared memory base is not 1024-byte aligned (the 128-byte swizzled TMA
+// tiles need it); it then returns without computing anything.
+constexpr int kErrSmemAlign = 6;
+
 // Forward, tensor-core path (bf16, B_q = B_k = 128).
 // Packed variable-length sequences (n = 0: fixed lengths, batch dimension
 // used instead). Sequence s owns query rows [q0[s], q0[s+1]) and key rows
@@ -102,7 +107,6 @@ cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
 struct BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;   // 4-D maps, box {64, 1, 128, 1}, 128B swizzle
   const float* zl2;        // [B, Hq, Npad] z log2e
-  const float* t2;         // [B, Hq, Npad] z + log tau - log L_q (natural log)
   const float* Dv;         // [B, Hq, Npad] rowsum(dO o O)
   float* dq_acc;           // [B, Hq, nQB, 32 column quads, 128 rows, 4] fp32
   void* dk;
@@ -118,6 +122,7 @@ struct BwdParams {
   uint8_t group_heads[kMaxKvHeads][kMaxGroup];
   SeqTable seq;            // packed sequences (B = their number; nQB / nKB maxima)
   uint64_t wait_ns;        // limit of every bounded wait (ns)
+  float log2_tau;          // log2(tau): -inf for tau = 0, +inf for tau = inf
 };
 
 struct BwdAuxParams {      // pre-pass and dQ conversion
@@ -125,14 +130,11 @@ struct BwdAuxParams {      // pre-pass and dQ conversion
   const void* dout;
   const float* lse;
   float* zl2;
-  float* t2;
   float* Dv;
   float* dq_acc;
   void* dq;
   int64_t o_sb, o_sn, o_sh, do_sb, do_sn, do_sh, dq_sb, dq_sn, dq_sh;
   int B, Hq, N, Npad, nQB;   // N = N_q
-  int q_off;                 // query q sits at position q + q_off: L_q = q + q_off + 1
-  float log_tau;
   SeqTable seq;              // packed sequences (B = their number)
 };
 

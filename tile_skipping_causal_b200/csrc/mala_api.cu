@@ -185,6 +185,8 @@ int mala_check_device_error(void* stream) {
   if (rec[0] != 0) {
     int zero[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     cudaMemcpyToSymbol(mala::g_device_error, zero, sizeof(zero));
+    if (rec[0] == mala::kErrSmemAlign)
+      return fail(MALA_ERR_CUDA, "a kernel found its dynamic shared memory base misaligned; nothing was computed");
     return fail(MALA_ERR_TIMEOUT,
                 "a device-side bounded wait gave up (role %d, barrier %d, tile %d, block %d, parity %d; "
                 "progress %08x %08x %08x)",
@@ -407,10 +409,10 @@ size_t bwd_rows(const mala_bwd_args* a) {
   return static_cast<size_t>(a->batch) * a->heads_q * npad;
 }
 
-// workspace: zl2, t2, D (one fp32 per row each) then the blocked dQ accumulator
+// workspace: zl2, D (one fp32 per row each) then the blocked dQ accumulator
 size_t bwd_ws_bytes(const mala_bwd_args* a) {
   const size_t rows = bwd_rows(a);
-  return rows * 3 * sizeof(float) + rows * 128 * sizeof(float) + 256;
+  return rows * 2 * sizeof(float) + rows * 128 * sizeof(float) + 256;
 }
 
 }  // namespace
@@ -454,14 +456,14 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
   if ((rc = make_map_bf16(&p.tm_do, a->dout, mb, N, a->heads_q, 128, a->do_stride, 128))) return rc;
   float* ws = static_cast<float*>(workspace);
   p.zl2 = ws;
-  p.t2 = ws + rows;
-  p.Dv = ws + 2 * rows;
-  p.dq_acc = ws + 3 * rows;
+  p.Dv = ws + rows;
+  p.dq_acc = ws + 2 * rows;
   p.dk = a->dk;
   p.dv = a->dv;
   p.fwd_mask = a->keep_mask;
   p.bwd_mask = a->bwd_keep_mask;
   p.stats = a->stats;
+  p.log2_tau = a->tau == 0.0f ? -INFINITY : log2f(a->tau);
   if ((rc = wait_limit(a->wait_limit_ns, &p.wait_ns))) return rc;
   p.err = device_error_ptr();
   if (!p.err) return fail(MALA_ERR_CUDA, "cannot resolve the device error word");
@@ -484,9 +486,8 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
   x.dout = a->dout;
   x.lse = a->lse;
   x.zl2 = ws;
-  x.t2 = ws + rows;
-  x.Dv = ws + 2 * rows;
-  x.dq_acc = ws + 3 * rows;
+  x.Dv = ws + rows;
+  x.dq_acc = ws + 2 * rows;
   x.dq = a->dq;
   x.o_sb = a->o_stride[0]; x.o_sn = a->o_stride[1]; x.o_sh = a->o_stride[2];
   x.do_sb = a->do_stride[0]; x.do_sn = a->do_stride[1]; x.do_sh = a->do_stride[2];
@@ -496,9 +497,7 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
   x.N = N;
   x.Npad = Npad;
   x.nQB = nQB;
-  x.q_off = Nk - N;
   x.seq = p.seq;
-  x.log_tau = a->tau == 0.0f ? -INFINITY : logf(a->tau);
 
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (a->bwd_keep_mask) {
