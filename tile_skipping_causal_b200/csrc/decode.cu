@@ -13,8 +13,7 @@
 // for tcgen05 (M >= 64), so scores and PV use warp-level mma.sync on
 // operands staged by TMA in 128-byte-swizzled shared memory.
 //
-// Roles (32 (W + 1) threads; W = 4 compute warps for bf16 caches, 8 for
-// e4m3 caches, whose per-tile work has more latency to hide):
+// Roles (32 (W + 1) threads; W = 4 compute warps):
 //   warps 0..W-1  compute. QK^T: warp w scores keys [w 128/W, (w+1) 128/W)
 //              of the tile for all rows; row maxima meet in shared memory;
 //              every warp then evaluates the same per-head decisions. PV:
@@ -27,9 +26,15 @@
 // one of two slots until the slot is needed again or the split ends, so the
 // V load issued after the decision overlaps the scoring of later tiles.
 //
-// FP8 (e4m3) caches: tiles arrive as 128-byte rows (half the bytes, so the
-// K ring is twice as deep), and the mma.sync B fragments are built straight
-// from them, converting in registers (exactly: every e4m3 value is an f16):
+// Residency: a bf16 CTA (4-tile K ring) fills an SM's shared memory. An
+// e4m3 tile has half the bytes but the same fragment work, so one CTA per
+// SM leaves the SM waiting on its per-tile chain; an e4m3 CTA instead keeps
+// a 2-tile K ring (76 KB of shared memory, 128 registers per thread) and
+// three CTAs share an SM, each streaming its own split.
+//
+// FP8 (e4m3) caches: tiles arrive as 128-byte rows, and the mma.sync B
+// fragments are built straight from them, converting in registers (exactly:
+// every e4m3 value is an f16):
 //   QK: the head dimension is visited in a permuted order, the same for the
 //       query fragments and K, chosen so that a thread's 32 values of a key
 //       row are 32 contiguous bytes (two 16-byte loads);
@@ -47,6 +52,15 @@
 #ifndef MALA_DECODE_BF16_WARPS
 #define MALA_DECODE_BF16_WARPS 4
 #endif
+#ifndef MALA_DECODE_FP8_WARPS
+#define MALA_DECODE_FP8_WARPS 4
+#endif
+#ifndef MALA_DECODE_FP8_RING
+#define MALA_DECODE_FP8_RING 2
+#endif
+#ifndef MALA_DECODE_FP8_CTAS
+#define MALA_DECODE_FP8_CTAS 3
+#endif
 
 namespace mala {
 
@@ -54,7 +68,7 @@ namespace {
 
 constexpr int kBK = 128;
 constexpr int kD = 128;
-constexpr int kNSKMax = 8;              // K ring stages: 4 bf16 tiles, 8 e4m3 tiles
+constexpr int kNSKMax = 8;              // K ring stages at most (4 bf16 tiles, 2 e4m3 tiles)
 constexpr int kNSV = 2;                 // V / P slots
 constexpr uint32_t kTileBytes = kBK * kD * 2;   // bf16 tile
 constexpr int kPStride = 136;           // bf16 per P row (128 + 8 padding)
@@ -72,11 +86,12 @@ enum Bar {
 
 template <bool FP8>
 struct Smem {
-  static constexpr int kCW = FP8 ? 8 : MALA_DECODE_BF16_WARPS;          // compute warps
+  static constexpr int kCW = FP8 ? MALA_DECODE_FP8_WARPS : MALA_DECODE_BF16_WARPS;   // compute warps
+  static constexpr int kMinCtas = FP8 ? MALA_DECODE_FP8_CTAS : 1;       // resident CTAs per SM
   static constexpr int kThreads = 32 * (kCW + 1);                       // + the producer warp
   static constexpr int kKPW = kBK / kCW;      // keys (scores) and value columns (PV) per compute warp
   static constexpr int kNBW = kKPW / 8;       // mma n-blocks per compute warp
-  static constexpr int kNSK = FP8 ? 8 : 4;                              // K ring stages
+  static constexpr int kNSK = FP8 ? MALA_DECODE_FP8_RING : 4;          // K ring stages
   static constexpr uint32_t kRing = FP8 ? kBK * kD : kTileBytes;        // bytes of a K / V ring tile
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + kNSK * kRing;
@@ -94,7 +109,7 @@ static_assert(Smem<false>::kPMax % 16 == 0 && Smem<true>::kPMax % 16 == 0, "per-
 static_assert(Smem<false>::kNSK <= kNSKMax && Smem<true>::kNSK <= kNSKMax, "K ring exceeds its barriers");
 
 template <bool FP8>
-__global__ void __launch_bounds__(Smem<FP8>::kThreads, 1) mala_decode_split_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(Smem<FP8>::kThreads, Smem<FP8>::kMinCtas) mala_decode_split_kernel(const __grid_constant__ DecodeParams p) {
   using Smem = mala::Smem<FP8>;
   constexpr uint32_t kRing = Smem::kRing;
   constexpr int kNSK = Smem::kNSK;
