@@ -55,7 +55,7 @@ struct Smem {
   static constexpr uint32_t kDO = kQ + 2 * kTile;
   static constexpr uint32_t kDS = kDO + kTile;
   static constexpr uint32_t kStage = kDS + kTile;           // dQ staging: 16 KB per compute warpgroup
-  static constexpr uint32_t kStats = kStage + kTile;        // [2 stages][zl2, D][128]
+  static constexpr uint32_t kStats = kStage + kTile;        // [2 stages][-z log2e, D][128]
   static constexpr uint32_t kBars = kStats + 2 * 2 * 128 * 4;
   static constexpr uint32_t kMisc = kBars + kNumBars * 8;
   static constexpr uint32_t kEnd = kMisc + 64;
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
           tma_load_4d(sQ + st * kTile + c * kChunk, &p.tm_q, &bars[kQFull + st], c * 64, h, qrow0 + i * kB, tb);
         const int64_t row0 = qblock_index(p.seq, p.Hq, p.nQB, b, h, i) * kB;
         float* sst = sStats + st * 256;
-        bulk_load(sst, p.zl2 + row0, 512, &bars[kQFull + st]);
+        bulk_load(sst, p.nzl2 + row0, 512, &bars[kQFull + st]);
         bulk_load(sst + 128, p.Dv + row0, 512, &bars[kQFull + st]);
         return true;
       };
@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       if (bar_or(1, 256, !okq || *abort_flag != 0) || qi == kEndMarker) break;
       const int i = static_cast<int>(qi);
       const int h = static_cast<int>(misc[6 + st]);
-      const float4* zl2_4 = reinterpret_cast<const float4*>(sStats + st * 256 + c0);
+      const float4* nz_4 = reinterpret_cast<const float4*>(sStats + st * 256 + c0);
       const float4* dv_4 = reinterpret_cast<const float4*>(sStats + st * 256 + 128 + c0);
       // test over this half of the S^T row, in log2 units: retain iff some
       // legal entry has u + log2 L_q >= log2 tau, with u = s log2 e - z log2 e
@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       // key rows past N_k) only occur in tiles whose last key lies beyond the
       // block's first query position; there they are set to -inf once, which
       // makes u = -inf: they drop out of the test and their P^T is exactly 0.
-      // Padded query columns carry z log2 e = +inf and drop out the same way.
+      // Padded query columns carry -z log2 e = -inf and drop out the same way.
       const bool oks = __all_sync(0xffffffffu, mbar_wait(&bars[kSFull], n & 1, abort_flag, p.err, wait_tag(0, kSFull, n), p.wait_ns));
       uint32_t sr[2][32];
       if (oks) {
@@ -455,15 +455,17 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
       for (int e = 0; e < 8; ++e) mu[e] = -INFINITY;
 #pragma unroll
       for (int x4 = 0; x4 < 16; ++x4) {
-        const float4 zv = zl2_4[x4];
-        const float zz[4] = {zv.x, zv.y, zv.z, zv.w};
+        const float4 zv = nz_4[x4];
+        const int x = 4 * x4;
+        float u[4];
+        fma2(u[0], u[1], __uint_as_float(sr[x >> 5][x & 31]), __uint_as_float(sr[x >> 5][(x + 1) & 31]), kLog2e,
+             kLog2e, zv.x, zv.y);
+        fma2(u[2], u[3], __uint_as_float(sr[x >> 5][(x + 2) & 31]), __uint_as_float(sr[x >> 5][(x + 3) & 31]), kLog2e,
+             kLog2e, zv.z, zv.w);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int x = 4 * x4 + e;
-          const float u = fmaf(__uint_as_float(sr[x >> 5][x & 31]), kLog2e, -zz[e]);
-          sr[x >> 5][x & 31] = __float_as_uint(u);
-          mu[x & 7] = fmaxf(mu[x & 7], u);
-        }
+        for (int e = 0; e < 4; ++e) sr[x >> 5][(x + e) & 31] = __float_as_uint(u[e]);
+        mu[x4 & 7] = max3(mu[x4 & 7], u[0], u[1]);
+        mu[x4 & 7] = max3(mu[x4 & 7], u[2], u[3]);
       }
       const float M = fmaxf(fmaxf(fmaxf(mu[0], mu[1]), fmaxf(mu[2], mu[3])),
                             fmaxf(fmaxf(mu[4], mu[5]), fmaxf(mu[6], mu[7])));
@@ -549,10 +551,10 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
           for (int e = 0; e < 4; e += 2) {
             const int x = 8 * u + 4 * e2 + e;
             const uint32_t w = pp[x >> 1];
-            const float p0 = __uint_as_float(w << 16);
-            const float p1 = __uint_as_float(w & 0xFFFF0000u);
-            const float d0 = p0 * (__uint_as_float(dp[x >> 5][x & 31]) - dd[e]);
-            const float d1 = p1 * (__uint_as_float(dp[(x + 1) >> 5][(x + 1) & 31]) - dd[e + 1]);
+            float t0, t1, d0, d1;
+            sub2(t0, t1, __uint_as_float(dp[x >> 5][x & 31]), __uint_as_float(dp[(x + 1) >> 5][(x + 1) & 31]), dd[e],
+                 dd[e + 1]);
+            mul2(d0, d1, __uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u), t0, t1);
             pk[2 * e2 + (e >> 1)] = pack_bf16x2(d0, d1);
           }
         }
@@ -625,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1) mala_bwd_tc_kernel(const __grid_c
   if (tid == 0 && *abort_flag) drain_pause_ns(50000);
 }
 
-// D = rowsum(dO o O), zl2 = z log2e; padded rows: zl2 = +inf, D = 0; zero
+// D = rowsum(dO o O), nzl2 = -z log2e; padded rows: nzl2 = -inf, D = 0; zero
 // the block's dQ accumulator.
 // Query block of an auxiliary CTA: blk = qblock_index(b, h, i); the
 // sequence's first query row, batch coordinate and length.
@@ -693,10 +695,10 @@ __global__ void __launch_bounds__(128) mala_bwd_pre_kernel(const __grid_constant
     const float z = p.seq.n == 0 ? p.lse[(static_cast<int64_t>(ab.b) * p.Hq + h) * p.N + q]
                                  : p.lse[static_cast<int64_t>(h) * p.seq.q0[p.seq.n] + qr];
     p.Dv[row] = acc;
-    p.zl2[row] = z * kLog2e;
+    p.nzl2[row] = -z * kLog2e;
   } else {
     p.Dv[row] = 0.0f;
-    p.zl2[row] = INFINITY;
+    p.nzl2[row] = -INFINITY;
   }
   float4* acc4 = reinterpret_cast<float4*>(p.dq_acc + static_cast<int64_t>(blk) * (kB * kD));
   for (int e = t; e < kB * kD / 4; e += 128) acc4[e] = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -390,9 +390,11 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       // row maximum of this half: eight independent chains, then a tree
       float mx[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(sr[0][e]);
+      for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
 #pragma unroll
-      for (int x = 8; x < 64; ++x) mx[x & 7] = fmaxf(mx[x & 7], __uint_as_float(sr[x >> 5][x & 31]));
+      for (int x = 0; x < 64; x += 2)
+        mx[(x >> 1) & 7] = max3(mx[(x >> 1) & 7], __uint_as_float(sr[x >> 5][x & 31]),
+                                __uint_as_float(sr[x >> 5][(x + 1) & 31]));
       const float pmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const int par = t & 1;
@@ -500,16 +502,20 @@ __global__ void __launch_bounds__(kThreads, 1) mala_fwd_tc_kernel(const __grid_c
       // columns [32g, 32g + 32); both groups finished reading S before the vote
       // rows without a legal key (padding) get P = 0 through m2 = +inf
       const float neg_m2 = has_key ? -m2 : -INFINITY;
-      float psum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      float psum[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};   // four pairs of partial sums
       uint32_t pk[32];
 #pragma unroll
       for (int x = 0; x < 64; x += 2) {
-        const float a = ex2_approx(fmaf(__uint_as_float(sr[x >> 5][x & 31]), kLog2e, neg_m2));
-        const float bb = ex2_approx(fmaf(__uint_as_float(sr[x >> 5][(x + 1) & 31]), kLog2e, neg_m2));
-        psum[(x >> 1) & 3] += a + bb;
+        float ea, eb;
+        fma2(ea, eb, __uint_as_float(sr[x >> 5][x & 31]), __uint_as_float(sr[x >> 5][(x + 1) & 31]), kLog2e, kLog2e,
+             neg_m2, neg_m2);
+        const float a = ex2_approx(ea);
+        const float bb = ex2_approx(eb);
+        const int q2 = 2 * ((x >> 1) & 3);
+        add2(psum[q2], psum[q2 + 1], psum[q2], psum[q2 + 1], a, bb);
         pk[x >> 1] = pack_bf16x2(a, bb);
       }
-      const float ps = (psum[0] + psum[1]) + (psum[2] + psum[3]);
+      const float ps = ((psum[0] + psum[1]) + (psum[2] + psum[3])) + ((psum[4] + psum[5]) + (psum[6] + psum[7]));
       tmem_st16(tmem + sb * 128 + lane_addr + g * 32, &pk[0]);
       tmem_st16(tmem + sb * 128 + lane_addr + g * 32 + 16, &pk[16]);
       xsum[(par * 2 + g) * 128 + r] = ps;

@@ -106,7 +106,7 @@ cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
 // Backward (bf16, d = 128, B_q = B_k = 128, N_q <= N_k bottom-right aligned).
 struct BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;   // 4-D maps, box {64, 1, 128, 1}, 128B swizzle
-  const float* zl2;        // [B, Hq, Npad] z log2e
+  const float* nzl2;       // [B, Hq, Npad] -z log2e
   const float* Dv;         // [B, Hq, Npad] rowsum(dO o O)
   float* dq_acc;           // [B, Hq, nQB, 32 column quads, 128 rows, 4] fp32
   void* dk;
@@ -129,7 +129,7 @@ struct BwdAuxParams {      // pre-pass and dQ conversion
   const void* o;
   const void* dout;
   const float* lse;
-  float* zl2;
+  float* nzl2;
   float* Dv;
   float* dq_acc;
   void* dq;

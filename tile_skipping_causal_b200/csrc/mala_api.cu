@@ -409,7 +409,7 @@ size_t bwd_rows(const mala_bwd_args* a) {
   return static_cast<size_t>(a->batch) * a->heads_q * npad;
 }
 
-// workspace: zl2, D (one fp32 per row each) then the blocked dQ accumulator
+// workspace: -z log2e, D (one fp32 per row each) then the blocked dQ accumulator
 size_t bwd_ws_bytes(const mala_bwd_args* a) {
   const size_t rows = bwd_rows(a);
   return rows * 2 * sizeof(float) + rows * 128 * sizeof(float) + 256;
@@ -455,7 +455,7 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
   if ((rc = make_map_bf16(&p.tm_v, a->v, mb, Nk, a->heads_kv, 128, a->v_stride, 128))) return rc;
   if ((rc = make_map_bf16(&p.tm_do, a->dout, mb, N, a->heads_q, 128, a->do_stride, 128))) return rc;
   float* ws = static_cast<float*>(workspace);
-  p.zl2 = ws;
+  p.nzl2 = ws;
   p.Dv = ws + rows;
   p.dq_acc = ws + 2 * rows;
   p.dk = a->dk;
@@ -485,7 +485,7 @@ int mala_bwd(const mala_bwd_args* a, void* workspace, size_t ws_bytes, void* str
   x.o = a->o;
   x.dout = a->dout;
   x.lse = a->lse;
-  x.zl2 = ws;
+  x.nzl2 = ws;
   x.Dv = ws + rows;
   x.dq_acc = ws + 2 * rows;
   x.dq = a->dq;
