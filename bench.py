@@ -119,10 +119,13 @@ def _dist_init():
 # key/value bytes (read once, so traffic grows with N_k; the split partials
 # are the same at both sizes). Set an entry to None when its kernel changes.
 NCU_TRAFFIC = {
-    "mala_bwd_tc_kernel": 8_766_994_688 + 4_450_865_152,
+    "mala_bwd_tc_kernel": 9_435_351_552 + 4_808_597_504,
     # decode, bf16 cache: the N_k = 8192 launch read 2,148,169,472 B (K and V
     # 2,147,483,648 B) and wrote 6,148,608 B; K and V grow 16x at 131072
     "mala_decode_split_kernel@131072": 16 * 2_147_483_648 + (2_148_169_472 - 2_147_483_648) + 6_148_608,
+    # decode, e4m3 cache: the N_k = 8192 launch read 1,074,353,408 B (K and V
+    # 1,073,741,824 B) and wrote 6,011,904 B; K and V grow 16x at 131072
+    "mala_decode_split_kernel@131072/e4m3": 16 * 1_073_741_824 + (1_074_353_408 - 1_073_741_824) + 6_011_904,
 }
 
 
