@@ -325,7 +325,9 @@ MALA_API const char* mala_last_error_message(void);
 /*
  * Synchronise `stream` and report a device-side failure recorded by any
  * kernel of this library since the previous call: MALA_ERR_TIMEOUT if a
- * bounded wait gave up, MALA_ERR_CUDA if the stream reports a CUDA error,
+ * bounded wait gave up; MALA_ERR_CUDA if the stream reports a CUDA error,
+ * or if the backward kernel found its dynamic shared memory base not
+ * 1024-byte aligned (its swizzled tiles need it; it then computes nothing);
  * else MALA_OK. Clears the recorded flag.
  */
 MALA_API int mala_check_device_error(void* stream);
