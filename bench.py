@@ -147,6 +147,13 @@ def whole_job_rate(units_per_rank: float, world: int, seconds: float) -> float:
     return units_per_rank * world / seconds
 
 
+def workload_config(B: int, Hq: int, Hkv: int, N: int, d: int) -> dict:
+    """The "config" object of both arms' JSON lines (the same workload)."""
+    return {"workload": WORKLOAD, "batch": B, "heads_q": Hq, "heads_kv": Hkv, "seqlen": N,
+            "head_dim": d, "block_q": TILE, "block_k": TILE, "tau": TAU, "pass": "fwd+bwd",
+            "l2": "inputs (0.7 GB) larger than L2; no flush"}
+
+
 def tile_flops(d: int = 128, bq: int = TILE, bk: int = TILE) -> float:
     """FLOPs of one bq x bk x d tile matmul (2 per multiply-add)."""
     return 2.0 * bq * bk * d
@@ -378,9 +385,7 @@ def run_mala(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic, seeded (gqa_32k recipe: diffuse / local / retrieval head thirds; dO ~ N(0,1))",
-        "config": {"workload": WORKLOAD, "batch": B, "heads_q": Hq, "heads_kv": Hkv, "seqlen": N,
-                   "head_dim": d, "block_q": TILE, "block_k": TILE, "tau": TAU, "pass": "fwd+bwd",
-                   "l2": "inputs (0.7 GB) larger than L2; no flush"},
+        "config": workload_config(B, Hq, Hkv, N, d),
         "tflops_executed": (fwd_flops + bwd_flops) / (elapsed / args.steps / world) / 1e12,
         "fwd": {"ms": kern_f * 1e3, "tflops_executed": ach_f, **tc_fracs(ach_f, peaks),
                 "tiles_tested": tested, "tiles_kept": kept, "kept_fraction": kept / tested,
@@ -748,6 +753,12 @@ def cpu_baseline(seconds: float = 15.0):
                       f"fp64 numpy, {secs:.1f} s"}
 
 
+def _reference_config() -> dict:
+    from tile_skipping_causal_b200 import synth
+    w = synth.WORKLOADS[WORKLOAD]
+    return workload_config(w.batch, w.heads_q, w.heads_kv, w.seqlen, w.head_dim)
+
+
 def run_reference(args):
     world, rank, _ = _dist_init()
     if rank != 0:
@@ -767,8 +778,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs_total / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic, seeded (gqa_32k recipe)",
-        "config": {"workload": WORKLOAD, "batch": 1, "heads_q": 32, "heads_kv": 8, "seqlen": 32768,
-                   "head_dim": 128, "block_q": TILE, "block_k": TILE, "tau": TAU, "pass": "fwd+bwd"},
+        "config": _reference_config(),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
                          "sample": f"{args.steps} steps of random 128-row query blocks, "
                                    f"{secs_total:.1f} s total"},
